@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Benchmark of the decode-attention hot path on B200.
+
+One step = one gqa_decode_attend call over the whole batch (split-KV partition
+kernel + merge/finalize kernel) on the 16-sequence bf16 workload: batch 16,
+32 Q / 8 KV heads, head_dim 128, 4096 cached keys per sequence, q/K/V iid
+N(0,1), bf16 output. Inputs are resident in HBM before the timed region; two
+copies of the 256 MiB cache are alternated so consecutive steps never read a
+cache the 126 MB L2 could still hold.
+
+Prints ONE JSON line (rank 0). `value` is the KV-cache bytes read per step,
+summed over ranks, divided by the max-over-ranks device time (GB/s); `e2e` is
+the same metric through the same public call when every step also copies its
+inputs from pinned host memory and its output back.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--no-cpu-baseline]
+
+--impl reference times the f64 CPU oracle (the library's reference
+implementation) on a bounded sample of the same workload, on rank 0 only.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GQA decode attention: KV-cache HBM GB/s (% of B200 peak) and queries·heads/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c2_bf16")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gqa_decode_attention_attend_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """dram read+write bytes per launch of the partition kernel from the committed
+    ncu summary, or None if there is none or the kernel sources changed since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return int(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline)
+
+def oracle_sample(w, seconds):
+    """Time the f64 oracle on whole copies of the workload until `seconds` pass.
+    Returns (GB/s, queries*heads/s, threads, sample description)."""
+    import oracle
+    from gqa_decode_attention_attend_b200 import workloads
+    q, k, v = (workloads.host_array(t) for t in (w.q, w.k, w.v))
+    off = w.offsets.numpy()
+    carry = tuple(t.numpy() for t in w.carry) if w.carry is not None else None
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_attend(q, k, v, off, w.num_heads, w.num_kv_heads, w.score_scale, carry=carry)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+    gbs = w.kv_bytes() * reps / dt / 1e9
+    qh = w.batch * w.num_heads * reps / dt
+    return gbs, qh, oracle.default_threads(), f"{reps} full passes of {w.name} ({dt:.1f} s wall)"
+
+
+# ------------------------------------------------------------------ ours
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import gqa_decode_attention_attend_b200 as gqa
+    from gqa_decode_attention_attend_b200 import workloads
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    w = workloads.config(args.workload)
+    if world > 1:
+        # weak scaling: every rank owns a different batch of the same shape
+        base = workloads.config(args.workload)
+        w = workloads.make(base.name, base.lengths, base.num_heads, base.num_kv_heads, base.head_dim,
+                           dtype=base.k.dtype, dist=base.meta["dist"], seed=1000 + rank,
+                           score_scale=base.score_scale, carry=base.carry is not None,
+                           needle=dict(amp=8.0, depth=4096) if base.meta["dist"] == "needle" else None)
+    H, G, D = w.num_heads, w.num_kv_heads, w.head_dim
+    kv_bytes = w.kv_bytes()
+    q = w.q.to(dev)
+    offsets = w.offsets.to(dev)
+    # two cache copies, alternated step by step (together > 2x L2)
+    caches = [(w.k.to(dev), w.v.to(dev))]
+    if kv_bytes < 4 * 126e6:
+        caches.append((caches[0][0].clone(), caches[0][1].clone()))
+    carry = gqa.State(*(t.to(dev) for t in w.carry)) if w.carry is not None else None
+    out = torch.empty(q.shape, dtype=q.dtype, device=dev)
+    ws = gqa.Workspace(dev)
+
+    def step(i):
+        k, v = caches[i % len(caches)]
+        gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
+                              out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    assert gqa.gqa_get_device_error(ws) == 0
+
+    sampler = ClockSampler(local) if rank == 0 or world > 1 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    # keep the same load for at least ~1.5 s so the clock sampler sees it
+    extra_t0 = time.perf_counter()
+    i = 0
+    while ms_total / 1e3 + (time.perf_counter() - extra_t0) < 1.5:
+        for _ in range(200):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = kv_bytes * world / (ms_per_step / 1e3) / 1e9
+
+    # ---- dominant kernel alone: the partition launch (partials-only call)
+    S_ws, S, chunk = gqa.gqa_decode_workspace_size(q, caches[0][0], caches[0][1], offsets, H, G,
+                                                   score_scale=w.score_scale, want_out=True,
+                                                   max_seq_len=w.max_seq_len)
+    parts = gqa.State.empty(w.batch * H, D, dev, (S,))
+
+    def part_only(i):
+        k, v = caches[i % len(caches)]
+        gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, partials_out=parts,
+                              num_splits=S, max_seq_len=w.max_seq_len, workspace=ws, stream=stream)
+
+    for i in range(5):
+        part_only(i)
+    n_part = max(args.steps, 50)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n_part):
+        part_only(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    part_ms = e0.elapsed_time(e1) / n_part
+    peak, peak_src = measured_peaks()
+    achieved = kv_bytes / (part_ms / 1e3) / 1e9
+
+    # ---- end to end: pinned host inputs -> device, call, output -> pinned host
+    hq = w.q.pin_memory()
+    hk = w.k.pin_memory()
+    hv = w.v.pin_memory()
+    hoff = w.offsets.pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dk, dv = caches[0]
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() * 2 + hoff.numel() * 4
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        offsets.copy_(hoff, non_blocking=True)
+        gqa.gqa_decode_attend(q, dk, dv, offsets, H, G, score_scale=w.score_scale, carry=carry, out=out,
+                              max_seq_len=w.max_seq_len, workspace=ws, stream=stream)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([x0.elapsed_time(x1) / args.e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+    e2e_value = kv_bytes * world / (e2e_ms / 1e3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, qh, cores, sample = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "queries_heads_per_s": qh}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if w.k.dtype == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded, no dataset)",
+            "config": {
+                "workload": w.name, "text": w.meta.get("text", ""), "batch": w.batch,
+                "num_heads": H, "num_kv_heads": G, "head_dim": D, "seq_len": w.max_seq_len,
+                "kv_bytes_per_step": kv_bytes, "num_splits": S, "chunk_len": chunk,
+                "l2": f"inputs larger than L2: {len(caches)} cache copies of {kv_bytes / 2**20:.0f} MiB alternated",
+                "parallelism": f"replicas x{world} (independent batches, no collective)",
+            },
+            "queries_heads_per_s": w.batch * H * world / (ms_per_step / 1e3),
+            "pct_of_nominal_8tbs": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
+            "pct_of_measured_peak": round(100.0 * value / world / peak, 2),
+            "roofline": {
+                "bound": "hbm", "kernel": "gqa_partition_bf16_kernel" if w.k.dtype == torch.bfloat16
+                else "gqa_partition_f32_kernel",
+                "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
+                "algorithmic_bytes_per_launch": kv_bytes, "launch_ms": part_ms,
+            },
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm (CPU oracle)
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from gqa_decode_attention_attend_b200 import workloads
+    import oracle
+    w = workloads.config(args.workload)
+    # each step: the oracle over a bounded sample of the workload (the first
+    # sequences of the batch, all their heads), sized to a few hundred ms
+    nseq = max(1, min(w.batch, 4))
+    o = w.offsets[: nseq + 1]
+    ws = workloads.make(w.name, w.lengths[:nseq], w.num_heads, w.num_kv_heads, w.head_dim,
+                        dtype=w.k.dtype, seed=0)
+    ws.q, ws.k, ws.v = w.q[:nseq], w.k[: int(o[-1])], w.v[: int(o[-1])]
+    ws.carry = None if w.carry is None else tuple(t[: nseq * w.num_heads] for t in w.carry)
+    ws.score_scale = w.score_scale
+    q, k, v = (workloads.host_array(t) for t in (ws.q, ws.k, ws.v))
+    off = ws.offsets.numpy()
+    carry = tuple(t.numpy() for t in ws.carry) if ws.carry is not None else None
+
+    def step():
+        oracle.decode_attend(q, k, v, off, w.num_heads, w.num_kv_heads, w.score_scale, carry=carry)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    steps = args.steps
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+        if time.perf_counter() - t0 > 120:        # keep the arm within a few minutes
+            steps = _ + 1
+            break
+    dt = (time.perf_counter() - t0) / steps
+    kvb = ws.kv_bytes()
+    value = kvb / dt / 1e9
+    cores = oracle.default_threads()
+    sample = f"first {nseq} of {w.batch} sequences of {w.name}, all heads ({kvb / 2**20:.0f} MiB KV)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded, no dataset)",
+        "config": {"workload": w.name, "text": w.meta.get("text", ""), "batch": w.batch,
+                   "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+                   "head_dim": w.head_dim, "seq_len": w.max_seq_len},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

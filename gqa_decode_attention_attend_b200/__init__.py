@@ -1,0 +1,354 @@
+"""Python binding of the B200 grouped-query decode-attention library.
+
+Thin ctypes marshalling over the C ABI declared in ``include/gqa_decode.h``:
+every step of the computation runs in the library's CUDA kernels. PyTorch
+provides device memory (the tensors passed in, and outputs/workspace allocated
+here when the caller gives none) and the current CUDA stream.
+
+The entry points keep the C names:
+  gqa_decode_attend, gqa_decode_workspace_size, gqa_workspace_init,
+  gqa_softmax_merge, gqa_state_finalize, gqa_get_device_error,
+  gqa_plan_splits, gqa_status_string, gqa_version.
+
+If the compiled library is missing the first call raises ``LibraryMissing``;
+there is no fallback implementation.
+"""
+import ctypes
+import math
+import os
+
+__all__ = [
+    "GqaError", "LibraryMissing", "State", "Workspace", "gqa_decode_attend",
+    "gqa_decode_workspace_size", "gqa_workspace_init", "gqa_softmax_merge", "gqa_state_finalize",
+    "gqa_get_device_error", "gqa_plan_splits", "gqa_status_string", "gqa_version", "lib_path",
+    "load_library",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "lib", "libgqa_decode.so")
+
+GQA_OK = 0
+GQA_ERR_INVALID_ARGUMENT = 1
+GQA_ERR_SHAPE_MISMATCH = 2
+GQA_ERR_DEVICE = 3
+GQA_ERR_WORKSPACE = 4
+GQA_ERR_BAD_OFFSETS = 5
+GQA_ERR_TIMEOUT = 6
+GQA_F32 = 0
+GQA_BF16 = 1
+
+
+class LibraryMissing(RuntimeError):
+    pass
+
+
+class GqaError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = int(status)
+        super().__init__(f"{where}: {gqa_status_string(self.status)} ({self.status})")
+
+
+class _CState(ctypes.Structure):
+    _fields_ = [("m", ctypes.c_void_p), ("l", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
+
+
+class _CParams(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32),
+        ("q", ctypes.c_void_p), ("q_dtype", ctypes.c_int32),
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("kv_dtype", ctypes.c_int32),
+        ("offsets", ctypes.c_void_p),
+        ("batch", ctypes.c_int32), ("max_len", ctypes.c_int32), ("max_seq_len", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("score_scale", ctypes.c_float),
+        ("carry_in", _CState), ("state_out", _CState),
+        ("out", ctypes.c_void_p), ("out_dtype", ctypes.c_int32),
+        ("partials_out", _CState),
+        ("num_splits", ctypes.c_int32),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+_lib = None
+
+
+def lib_path():
+    return _LIB_PATH
+
+
+def load_library(path=None):
+    """Load libgqa_decode.so (once). Raises LibraryMissing if it was never built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise LibraryMissing(
+            f"{p} not found: build it with `python -m gqa_decode_attention_attend_b200.build`")
+    lib = ctypes.CDLL(p)
+    sp = ctypes.c_void_p
+    i32, i64 = ctypes.c_int32, ctypes.c_int64
+    ps = ctypes.POINTER(_CState)
+    lib.gqa_decode_workspace_size.argtypes = [ctypes.POINTER(_CParams), ctypes.POINTER(ctypes.c_size_t),
+                                              ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.gqa_workspace_init.argtypes = [sp, ctypes.c_size_t, sp]
+    lib.gqa_decode_attend.argtypes = [ctypes.POINTER(_CParams), sp]
+    lib.gqa_softmax_merge.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
+    lib.gqa_state_finalize.argtypes = [ps, i32, i32, sp, i32, sp]
+    lib.gqa_get_device_error.argtypes = [sp, sp]
+    lib.gqa_plan_splits.argtypes = [i32, i32, i32, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.gqa_status_string.argtypes = [ctypes.c_int]
+    lib.gqa_status_string.restype = ctypes.c_char_p
+    lib.gqa_version.argtypes = []
+    for fn in ("gqa_decode_workspace_size", "gqa_workspace_init", "gqa_decode_attend", "gqa_softmax_merge",
+               "gqa_state_finalize", "gqa_get_device_error", "gqa_plan_splits"):
+        getattr(lib, fn).restype = ctypes.c_int
+    lib.gqa_version.restype = ctypes.c_int32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def gqa_status_string(status):
+    return load_library().gqa_status_string(int(status)).decode()
+
+
+def gqa_version():
+    return int(load_library().gqa_version())
+
+
+def _check(status, where):
+    if status != GQA_OK:
+        raise GqaError(status, where)
+
+
+# ------------------------------------------------------------------ torch marshalling
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return GQA_F32
+    if t.dtype == torch.bfloat16:
+        return GQA_BF16
+    raise GqaError(GQA_ERR_SHAPE_MISMATCH, f"dtype {t.dtype}")
+
+
+def _torch_dtype(code):
+    torch = _torch()
+    return torch.bfloat16 if code == GQA_BF16 else torch.float32
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise GqaError(GQA_ERR_INVALID_ARGUMENT, "tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class State:
+    """An online-softmax state (m [n], l [n], acc [n, D]) of fp32 device tensors."""
+
+    def __init__(self, m, l, acc):
+        self.m, self.l, self.acc = m, l, acc
+
+    @classmethod
+    def empty(cls, rows, head_dim, device, extra=()):
+        torch = _torch()
+        shape = (rows, *extra)
+        return cls(torch.empty(shape, dtype=torch.float32, device=device),
+                   torch.empty(shape, dtype=torch.float32, device=device),
+                   torch.empty((*shape, head_dim), dtype=torch.float32, device=device))
+
+    def _c(self):
+        return _CState(_ptr(self.m), _ptr(self.l), _ptr(self.acc))
+
+
+def _c_state(s):
+    return _CState(None, None, None) if s is None else s._c()
+
+
+class Workspace:
+    """Scratch memory for gqa_decode_attend: a uint8 device tensor, 256-byte
+    aligned, whose error word is zeroed once by gqa_workspace_init. It grows on
+    demand (and is then re-initialised)."""
+
+    def __init__(self, device, nbytes=256):
+        self.device = device
+        self.tensor = None
+        self.reserve(nbytes)
+
+    def reserve(self, nbytes, stream=None):
+        torch = _torch()
+        if self.tensor is not None and self.tensor.numel() >= nbytes + 256:
+            return
+        n = max(int(nbytes), 256) + 256
+        self.tensor = torch.empty(n, dtype=torch.uint8, device=self.device)
+        _check(load_library().gqa_workspace_init(ctypes.c_void_p(self.ptr), self.nbytes,
+                                                 _stream_handle(stream)), "gqa_workspace_init")
+
+    @property
+    def ptr(self):
+        p = self.tensor.data_ptr()
+        return (p + 255) & ~255
+
+    @property
+    def nbytes(self):
+        return self.tensor.numel() - (self.ptr - self.tensor.data_ptr())
+
+
+_default_ws = {}
+
+
+def _default_workspace(device):
+    key = str(device)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out,
+            out_dtype, partials_out, num_splits, max_seq_len, max_len):
+    p = _CParams()
+    p.struct_size = ctypes.sizeof(_CParams)
+    p.q, p.q_dtype = _ptr(q), _dtype_code(q)
+    p.k, p.v, p.kv_dtype = _ptr(k), _ptr(v), _dtype_code(k)
+    if v.dtype != k.dtype:
+        raise GqaError(GQA_ERR_SHAPE_MISMATCH, "k and v dtypes differ")
+    p.offsets = _ptr(offsets)
+    p.batch = offsets.numel() - 1
+    p.max_len = k.shape[0] if max_len is None else int(max_len)
+    p.max_seq_len = int(max_seq_len)
+    p.num_heads = int(num_heads)
+    p.num_kv_heads = int(num_kv_heads)
+    p.head_dim = q.shape[-1]
+    p.score_scale = float(score_scale)
+    p.carry_in = _c_state(carry)
+    p.state_out = _c_state(state_out)
+    p.out = _ptr(out)
+    p.out_dtype = out_dtype
+    p.partials_out = _c_state(partials_out)
+    p.num_splits = int(num_splits)
+    return p
+
+
+def gqa_decode_workspace_size(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scale=0.0,
+                              carry=None, state_out=None, want_out=True, partials_out=None,
+                              num_splits=0, max_seq_len=0, max_len=None):
+    """(bytes, num_splits, chunk_len) the library will use for such a call."""
+    torch = _torch()
+    # sizing never dereferences out; a one-element placeholder marks it as wanted
+    placeholder = torch.empty(1, dtype=q.dtype, device=q.device) if want_out else None
+    p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out,
+                placeholder, _dtype_code(q), partials_out, num_splits, max_seq_len, max_len)
+    nbytes = ctypes.c_size_t()
+    ns = ctypes.c_int32()
+    cl = ctypes.c_int32()
+    _check(load_library().gqa_decode_workspace_size(ctypes.byref(p), ctypes.byref(nbytes),
+                                                    ctypes.byref(ns), ctypes.byref(cl)),
+           "gqa_decode_workspace_size")
+    return nbytes.value, ns.value, cl.value
+
+
+def gqa_decode_attend(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scale=0.0, carry=None,
+                      state_out=None, out=None, out_dtype=None, partials_out=None, want_out=None,
+                      num_splits=0, max_seq_len=0, max_len=None, workspace=None, stream=None):
+    """Decode attention over a KV cache; see include/gqa_decode.h.
+
+    q [B, H, D]; k, v [max_len, G, D]; offsets int32 [B+1] on the device.
+    carry / state_out / partials_out: ``State`` objects or None. ``out`` is
+    allocated ([B, H, D], out_dtype or q's dtype) unless given, or unless only
+    state_out / partials_out are wanted (want_out=False). Returns out (or None).
+    """
+    torch = _torch()
+    if want_out is None:
+        want_out = out is not None or (state_out is None and partials_out is None)
+    odt = _dtype_code(q) if out_dtype is None else (out_dtype if isinstance(out_dtype, int)
+                                                    else _dtype_code(torch.empty(0, dtype=out_dtype)))
+    if want_out and out is None:
+        out = torch.empty(q.shape, dtype=_torch_dtype(odt), device=q.device)
+    if out is not None:
+        odt = _dtype_code(out)
+    p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
+                partials_out, num_splits, max_seq_len, max_len)
+    lib = load_library()
+    nbytes = ctypes.c_size_t()
+    _check(lib.gqa_decode_workspace_size(ctypes.byref(p), ctypes.byref(nbytes), None, None),
+           "gqa_decode_workspace_size")
+    ws = workspace or _default_workspace(q.device)
+    ws.reserve(nbytes.value, stream)
+    p.workspace = ws.ptr
+    p.workspace_bytes = ws.nbytes
+    _check(lib.gqa_decode_attend(ctypes.byref(p), _stream_handle(stream)), "gqa_decode_attend")
+    return out
+
+
+def gqa_softmax_merge(states, carry=None, merged_out=None, out=None, out_dtype=None, want_out=None,
+                      stream=None):
+    """Merge states (m, l [rows, S]; acc [rows, S, D]) with an optional carry.
+    Returns out [rows, D] (allocated unless given or want_out=False)."""
+    torch = _torch()
+    rows, S = states.m.shape
+    D = states.acc.shape[-1]
+    if want_out is None:
+        want_out = out is not None or merged_out is None
+    if want_out and out is None:
+        out = torch.empty((rows, D), dtype=out_dtype or torch.float32, device=states.m.device)
+    odt = _dtype_code(out) if out is not None else GQA_F32
+    cs = states._c()
+    cc = _c_state(carry)
+    cm = _c_state(merged_out)
+    _check(load_library().gqa_softmax_merge(ctypes.byref(cs), rows, S, D, ctypes.byref(cc),
+                                            ctypes.byref(cm), _ptr(out), odt, _stream_handle(stream)),
+           "gqa_softmax_merge")
+    return out
+
+
+def gqa_state_finalize(state, out=None, out_dtype=None, stream=None):
+    """out = acc / l for a state (m, l [rows]; acc [rows, D])."""
+    torch = _torch()
+    rows = state.m.shape[0]
+    D = state.acc.shape[-1]
+    if out is None:
+        out = torch.empty((rows, D), dtype=out_dtype or torch.float32, device=state.m.device)
+    cs = state._c()
+    _check(load_library().gqa_state_finalize(ctypes.byref(cs), rows, D, _ptr(out), _dtype_code(out),
+                                             _stream_handle(stream)), "gqa_state_finalize")
+    return out
+
+
+def gqa_get_device_error(workspace=None, device=None, stream=None):
+    """Synchronise and return (and clear) the workspace's device error status."""
+    ws = workspace or _default_workspace(device if device is not None else _torch().device("cuda"))
+    return load_library().gqa_get_device_error(ctypes.c_void_p(ws.ptr), _stream_handle(stream))
+
+
+def gqa_workspace_init(workspace, stream=None):
+    _check(load_library().gqa_workspace_init(ctypes.c_void_p(workspace.ptr), workspace.nbytes,
+                                             _stream_handle(stream)), "gqa_workspace_init")
+
+
+def gqa_plan_splits(batch, num_kv_heads, max_seq_len, total_rows, resident_ctas):
+    """(chunk_len, num_splits) of the library's split heuristic (host only)."""
+    c = ctypes.c_int32()
+    s = ctypes.c_int32()
+    _check(load_library().gqa_plan_splits(int(batch), int(num_kv_heads), int(max_seq_len),
+                                          int(total_rows), int(resident_ctas), ctypes.byref(c),
+                                          ctypes.byref(s)), "gqa_plan_splits")
+    return c.value, s.value
+
+
+def default_scale(head_dim):
+    return 1.0 / math.sqrt(head_dim)

@@ -1,0 +1,518 @@
+// gqa_decode.cu -- C ABI of the decode-attention library (include/gqa_decode.h):
+// argument validation, the split heuristic, workspace sizing, TMA descriptor
+// encoding and the kernel launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/gqa_decode.h"
+#include "kernels.cuh"
+
+namespace {
+
+using gqa::MergeArgs;
+using gqa::PartitionArgs;
+
+constexpr int kVersion = 100;          // 0.1.0
+constexpr size_t kHeaderBytes = 256;   // error word + reserved
+constexpr int kChunkQuantum = 64;      // rows per pipeline stage of the bf16 kernel
+constexpr int kMaxHeadsPerKv = 16;
+constexpr int kMaxDevices = 64;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ------------------------------------------------------------------ device info
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+  int resident_bf16[2][2] = {{0, 0}, {0, 0}};   // [D==128][NT-1]
+  int resident_f32[2] = {0, 0};                 // [D==128], HMAX=16 worst case
+  cudaError_t err = cudaSuccess;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+template <int D, int NT>
+cudaError_t prepare_bf16(int* resident) {
+  using C = gqa::TcCfg<D, NT>;
+  cudaError_t e = cudaFuncSetAttribute(gqa::gqa_partition_bf16_kernel<D, NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(resident, gqa::gqa_partition_bf16_kernel<D, NT>,
+                                                       C::kThreads, C::kSmemBytes);
+}
+
+template <int D, int HMAX>
+cudaError_t prepare_f32(int* resident) {
+  using C = gqa::F32Cfg<D, HMAX>;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(resident, gqa::gqa_partition_f32_kernel<D, HMAX>,
+                                                       C::kThreads, C::kSmemBytes);
+}
+
+// Per-device one-time set-up (kernel attributes, occupancy, SM count).
+const DeviceInfo* device_info(int* dev_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (di.ready) return &di;
+  cudaDeviceProp prop;
+  cudaError_t e = cudaGetDeviceProperties(&prop, dev);
+  if (e == cudaSuccess && prop.major < 10) e = cudaErrorInvalidDevice;   // sm_100a code only
+  if (e == cudaSuccess) e = prepare_bf16<64, 1>(&di.resident_bf16[0][0]);
+  if (e == cudaSuccess) e = prepare_bf16<64, 2>(&di.resident_bf16[0][1]);
+  if (e == cudaSuccess) e = prepare_bf16<128, 1>(&di.resident_bf16[1][0]);
+  if (e == cudaSuccess) e = prepare_bf16<128, 2>(&di.resident_bf16[1][1]);
+  if (e == cudaSuccess) e = prepare_f32<64, 16>(&di.resident_f32[0]);
+  if (e == cudaSuccess) e = prepare_f32<128, 16>(&di.resident_f32[1]);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    di.err = e;
+    return nullptr;
+  }
+  di.sm_count = prop.multiProcessorCount;
+  di.ready = true;
+  return &di;
+}
+
+// ------------------------------------------------------------------ driver entry point
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// K or V cache [max_len, G, D] bf16 as a 2-D tensor (G*D columns, max_len rows);
+// box = 64 columns (128 bytes, one swizzle span) x 64 rows.
+bool make_kv_map(CUtensorMap* m, const void* base, int max_len, int G, int D) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(G) * D, static_cast<cuuint64_t>(max_len)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(G) * D * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kChunkQuantum)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ validation helpers
+
+bool is_device_ptr(const void* p) {
+  if (p == nullptr) return true;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+bool state_present(const gqa_state& s) { return s.m || s.l || s.acc; }
+bool state_complete(const gqa_state& s) { return s.m && s.l && s.acc; }
+
+struct Resolved {
+  int B, H, G, hpk, D, max_len, max_seq_len;
+  bool bf16;
+  int out_bf16;
+  float scale;
+  bool want_merge;      // out or state_out requested
+  bool has_partials;    // caller's partials_out
+  int S, chunk;         // split plan
+  int resident;         // partition CTAs resident on the whole GPU
+  size_t bytes;         // workspace bytes
+  size_t off_m, off_l, off_acc;
+};
+
+int nt_of(int hpk) { return hpk <= 8 ? 1 : 2; }
+
+gqa_status plan_impl(int32_t batch, int32_t G, int32_t max_seq_len, int64_t total_rows,
+                     int32_t resident, int32_t* chunk_len, int32_t* num_splits) {
+  if (batch < 0 || G <= 0 || max_seq_len < 0 || resident <= 0 || !chunk_len || !num_splits)
+    return GQA_ERR_INVALID_ARGUMENT;
+  if (max_seq_len == 0 || batch == 0) {
+    *chunk_len = kChunkQuantum;
+    *num_splits = 1;
+    return GQA_OK;
+  }
+  const int64_t full = static_cast<int64_t>(batch) * max_seq_len;
+  if (total_rows <= 0 || total_rows > full) total_rows = full;
+  const bool uniform = total_rows == full;
+  // Target enough CTAs that every SM holds several from the start and the last
+  // ones are short: 2 x resident for equal-length sequences, 8 x resident for a
+  // ragged batch (where chunk lengths vary).
+  const int64_t target = static_cast<int64_t>(resident) * (uniform ? 2 : 8);
+  const int64_t units = total_rows * G;                          // (row, KV head) pairs
+  int64_t chunk = (units + target - 1) / target;
+  const int64_t cap = (static_cast<int64_t>(max_seq_len) + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum;
+  chunk = (chunk + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum;
+  if (chunk < 4 * kChunkQuantum) chunk = 4 * kChunkQuantum;      // amortise the per-CTA prologue
+  if (chunk > cap) chunk = cap;
+  int64_t splits = (max_seq_len + chunk - 1) / chunk;
+  // even out the splits of a full-length sequence
+  chunk = ((max_seq_len + splits - 1) / splits + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum;
+  splits = (max_seq_len + chunk - 1) / chunk;
+  *chunk_len = static_cast<int32_t>(chunk);
+  *num_splits = static_cast<int32_t>(splits);
+  return GQA_OK;
+}
+
+// Host-side validation and planning shared by workspace_size and attend.
+gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
+  if (!p || p->struct_size != sizeof(gqa_decode_params)) return GQA_ERR_INVALID_ARGUMENT;
+  r->B = p->batch;
+  r->H = p->num_heads;
+  r->G = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
+  r->D = p->head_dim;
+  r->max_len = p->max_len;
+  if (r->B < 0 || r->H <= 0 || r->G <= 0 || r->H % r->G != 0) return GQA_ERR_INVALID_ARGUMENT;
+  r->hpk = r->H / r->G;
+  if (r->hpk > kMaxHeadsPerKv) return GQA_ERR_INVALID_ARGUMENT;
+  if (r->D != 64 && r->D != 128) return GQA_ERR_INVALID_ARGUMENT;
+  if (r->max_len < 0 || p->max_seq_len < 0 || p->num_splits < 0) return GQA_ERR_INVALID_ARGUMENT;
+  r->max_seq_len = p->max_seq_len == 0 ? r->max_len : p->max_seq_len;
+  if (r->max_seq_len > r->max_len) r->max_seq_len = r->max_len;
+  // q and an output are needed only when there is a sequence; K and V only
+  // when the cache has rows (an empty tensor may have a null data pointer).
+  if (!p->offsets) return GQA_ERR_INVALID_ARGUMENT;
+  if (r->B > 0 && !p->q) return GQA_ERR_INVALID_ARGUMENT;
+  if (r->max_len > 0 && (!p->k || !p->v)) return GQA_ERR_INVALID_ARGUMENT;
+  const bool has_carry = state_present(p->carry_in);
+  const bool has_state_out = state_present(p->state_out);
+  r->has_partials = state_present(p->partials_out);
+  if ((has_carry && !state_complete(p->carry_in)) || (has_state_out && !state_complete(p->state_out)) ||
+      (r->has_partials && !state_complete(p->partials_out)))
+    return GQA_ERR_INVALID_ARGUMENT;
+  if (r->B > 0 && !p->out && !has_state_out && !r->has_partials) return GQA_ERR_INVALID_ARGUMENT;
+  r->want_merge = p->out || has_state_out;
+  if (p->q_dtype != GQA_F32 && p->q_dtype != GQA_BF16) return GQA_ERR_SHAPE_MISMATCH;
+  if (p->kv_dtype != GQA_F32 && p->kv_dtype != GQA_BF16) return GQA_ERR_SHAPE_MISMATCH;
+  if (p->q_dtype != p->kv_dtype) return GQA_ERR_SHAPE_MISMATCH;
+  if (p->out && p->out_dtype != GQA_F32 && p->out_dtype != GQA_BF16) return GQA_ERR_SHAPE_MISMATCH;
+  r->bf16 = p->kv_dtype == GQA_BF16;
+  r->out_bf16 = p->out_dtype == GQA_BF16 ? 1 : 0;
+  const uintptr_t align_or = reinterpret_cast<uintptr_t>(p->q) | reinterpret_cast<uintptr_t>(p->k) |
+                             reinterpret_cast<uintptr_t>(p->v);
+  if (align_or & 15u) return GQA_ERR_SHAPE_MISMATCH;
+  if (!std::isfinite(p->score_scale)) return GQA_ERR_INVALID_ARGUMENT;
+  r->scale = p->score_scale != 0.f ? p->score_scale : 1.0f / sqrtf(static_cast<float>(r->D));
+  if (static_cast<int64_t>(r->B) * r->H * r->D > INT32_MAX) return GQA_ERR_INVALID_ARGUMENT;
+
+  r->resident = 0;
+  if (need_device) {
+    int dev;
+    const DeviceInfo* di = device_info(&dev);
+    if (!di) return GQA_ERR_DEVICE;
+    const int per_sm = r->bf16 ? di->resident_bf16[r->D == 128][nt_of(r->hpk) - 1]
+                               : di->resident_f32[r->D == 128];
+    r->resident = di->sm_count * (per_sm > 0 ? per_sm : 1);
+  }
+  // split plan
+  if (p->num_splits > 0) {
+    r->S = p->num_splits;
+    int64_t chunk = r->max_seq_len == 0 ? kChunkQuantum : (static_cast<int64_t>(r->max_seq_len) + r->S - 1) / r->S;
+    chunk = (chunk + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum;
+    r->chunk = static_cast<int>(chunk);
+  } else {
+    int32_t c, s;
+    const int64_t rows_hint = r->max_len;
+    gqa_status st = plan_impl(r->B, r->G, r->max_seq_len, rows_hint, r->resident > 0 ? r->resident : 296, &c, &s);
+    if (st != GQA_OK) return st;
+    r->S = s;
+    r->chunk = c;
+  }
+  if (static_cast<int64_t>(r->B) * r->S * r->G > INT32_MAX) return GQA_ERR_INVALID_ARGUMENT;
+  // workspace: header, then internal partial states when merging without the caller's
+  r->bytes = kHeaderBytes;
+  r->off_m = r->off_l = r->off_acc = 0;
+  if (r->want_merge && !r->has_partials) {
+    const size_t n = static_cast<size_t>(r->B) * r->H * r->S;
+    r->off_m = r->bytes;
+    r->bytes += align256(n * sizeof(float));
+    r->off_l = r->bytes;
+    r->bytes += align256(n * sizeof(float));
+    r->off_acc = r->bytes;
+    r->bytes += align256(n * r->D * sizeof(float));
+  }
+  return GQA_OK;
+}
+
+template <int D>
+cudaError_t launch_merge(const MergeArgs& m, cudaStream_t st) {
+  if (m.rows == 0) return cudaSuccess;
+  gqa::gqa_merge_kernel<D><<<m.rows, 128, 0, st>>>(m);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_any(int D, const MergeArgs& m, cudaStream_t st) {
+  return D == 128 ? launch_merge<128>(m, st) : launch_merge<64>(m, st);
+}
+
+template <int D, int NT>
+cudaError_t launch_bf16(const PartitionArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                        unsigned grid, cudaStream_t st) {
+  using C = gqa::TcCfg<D, NT>;
+  gqa::gqa_partition_bf16_kernel<D, NT><<<grid, C::kThreads, C::kSmemBytes, st>>>(tk, tv, a);
+  return cudaGetLastError();
+}
+
+template <int D, int HMAX>
+cudaError_t launch_f32(const PartitionArgs& a, unsigned grid, cudaStream_t st) {
+  using C = gqa::F32Cfg<D, HMAX>;
+  gqa::gqa_partition_f32_kernel<D, HMAX><<<grid, C::kThreads, C::kSmemBytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_partition(const Resolved& r, const PartitionArgs& a, const CUtensorMap* tk,
+                             const CUtensorMap* tv, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(r.B) * r.S * r.G;
+  if (grid == 0) return cudaSuccess;
+  if (r.bf16) {
+    const int nt = nt_of(r.hpk);
+    if (r.D == 128) return nt == 1 ? launch_bf16<128, 1>(a, *tk, *tv, grid, st) : launch_bf16<128, 2>(a, *tk, *tv, grid, st);
+    return nt == 1 ? launch_bf16<64, 1>(a, *tk, *tv, grid, st) : launch_bf16<64, 2>(a, *tk, *tv, grid, st);
+  }
+  if (r.D == 128) {
+    if (r.hpk <= 4) return launch_f32<128, 4>(a, grid, st);
+    if (r.hpk <= 8) return launch_f32<128, 8>(a, grid, st);
+    return launch_f32<128, 16>(a, grid, st);
+  }
+  if (r.hpk <= 4) return launch_f32<64, 4>(a, grid, st);
+  if (r.hpk <= 8) return launch_f32<64, 8>(a, grid, st);
+  return launch_f32<64, 16>(a, grid, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gqa_status_string(gqa_status s) {
+  switch (s) {
+    case GQA_OK: return "GQA_OK";
+    case GQA_ERR_INVALID_ARGUMENT: return "GQA_ERR_INVALID_ARGUMENT";
+    case GQA_ERR_SHAPE_MISMATCH: return "GQA_ERR_SHAPE_MISMATCH";
+    case GQA_ERR_DEVICE: return "GQA_ERR_DEVICE";
+    case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE";
+    case GQA_ERR_BAD_OFFSETS: return "GQA_ERR_BAD_OFFSETS";
+    case GQA_ERR_TIMEOUT: return "GQA_ERR_TIMEOUT";
+  }
+  return "GQA_ERR_UNKNOWN";
+}
+
+int32_t gqa_version(void) { return kVersion; }
+
+gqa_status gqa_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len, int64_t total_rows,
+                           int32_t resident_ctas, int32_t* chunk_len, int32_t* num_splits) {
+  return plan_impl(batch, num_kv_heads, max_seq_len, total_rows, resident_ctas, chunk_len, num_splits);
+}
+
+gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes, int32_t* num_splits,
+                                     int32_t* chunk_len) {
+  Resolved r;
+  gqa_status st = resolve(params, &r, true);
+  if (st != GQA_OK) return st;
+  if (bytes) *bytes = r.bytes;
+  if (num_splits) *num_splits = r.S;
+  if (chunk_len) *chunk_len = r.chunk;
+  return GQA_OK;
+}
+
+gqa_status gqa_workspace_init(void* workspace, size_t workspace_bytes, gqa_stream_t stream) {
+  if (!workspace || workspace_bytes < kHeaderBytes) return GQA_ERR_WORKSPACE;
+  if (!is_device_ptr(workspace)) return GQA_ERR_DEVICE;
+  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  return GQA_OK;
+}
+
+gqa_status gqa_decode_attend(const gqa_decode_params* p, gqa_stream_t stream) {
+  Resolved r;
+  gqa_status st = resolve(p, &r, true);
+  if (st != GQA_OK) return st;
+  if (!p->workspace || p->workspace_bytes < r.bytes) return GQA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
+  const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out, p->workspace,
+                        p->carry_in.m, p->carry_in.l, p->carry_in.acc,
+                        p->state_out.m, p->state_out.l, p->state_out.acc,
+                        p->partials_out.m, p->partials_out.l, p->partials_out.acc};
+  for (const void* q : ptrs)
+    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
+  if (r.B == 0) return GQA_OK;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  PartitionArgs a;
+  a.q = p->q;
+  a.k = p->k;
+  a.v = p->v;
+  a.offsets = p->offsets;
+  a.B = r.B;
+  a.H = r.H;
+  a.G = r.G;
+  a.hpk = r.hpk;
+  a.max_len = r.max_len;
+  a.chunk_len = r.chunk;
+  a.num_splits = r.S;
+  a.scale_log2 = r.scale * gqa::kLog2e;
+  if (r.has_partials) {
+    a.part_m = p->partials_out.m;
+    a.part_l = p->partials_out.l;
+    a.part_acc = p->partials_out.acc;
+    a.write_empty = 1;
+  } else {
+    a.part_m = reinterpret_cast<float*>(ws + r.off_m);
+    a.part_l = reinterpret_cast<float*>(ws + r.off_l);
+    a.part_acc = reinterpret_cast<float*>(ws + r.off_acc);
+    a.write_empty = 0;
+  }
+  a.err = reinterpret_cast<uint32_t*>(ws);
+
+  if (r.max_len > 0 || r.has_partials) {
+    // With no cache rows every tile is empty and no load is issued, but a
+    // tensor map still needs a non-zero extent and a valid aligned base: the
+    // workspace stands in for the (possibly null) empty caches.
+    CUtensorMap tk, tv;
+    const int map_rows = r.max_len > 0 ? r.max_len : 1;
+    const void* kb = r.max_len > 0 ? p->k : p->workspace;
+    const void* vb = r.max_len > 0 ? p->v : p->workspace;
+    if (r.bf16 && (!make_kv_map(&tk, kb, map_rows, r.G, r.D) || !make_kv_map(&tv, vb, map_rows, r.G, r.D)))
+      return GQA_ERR_DEVICE;
+    if (launch_partition(r, a, &tk, &tv, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+  }
+
+  if (r.want_merge) {
+    MergeArgs m;
+    m.m = a.part_m;
+    m.l = a.part_l;
+    m.acc = a.part_acc;
+    m.rows = r.B * r.H;
+    m.S = r.S;
+    m.offsets = p->offsets;
+    m.H = r.H;
+    m.chunk_len = r.chunk;
+    m.max_len = r.max_len;
+    const bool has_carry = state_present(p->carry_in);
+    m.cm = has_carry ? p->carry_in.m : nullptr;
+    m.cl = has_carry ? p->carry_in.l : nullptr;
+    m.cacc = has_carry ? p->carry_in.acc : nullptr;
+    const bool has_so = state_present(p->state_out);
+    m.om = has_so ? p->state_out.m : nullptr;
+    m.ol = has_so ? p->state_out.l : nullptr;
+    m.oacc = has_so ? p->state_out.acc : nullptr;
+    m.out = p->out;
+    m.out_bf16 = r.out_bf16;
+    if (launch_merge_any(r.D, m, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+  }
+  return GQA_OK;
+}
+
+static gqa_status merge_common(const gqa_state* states, int32_t rows, int32_t num_states, int32_t head_dim,
+                               const gqa_state* carry_in, const gqa_state* merged_out, void* out,
+                               int32_t out_dtype, gqa_stream_t stream) {
+  if (rows < 0 || num_states < 0 || (head_dim != 64 && head_dim != 128)) return GQA_ERR_INVALID_ARGUMENT;
+  if (num_states > 0 && (!states || !state_complete(*states))) return GQA_ERR_INVALID_ARGUMENT;
+  const bool has_carry = carry_in && state_present(*carry_in);
+  const bool has_out_state = merged_out && state_present(*merged_out);
+  if ((has_carry && !state_complete(*carry_in)) || (has_out_state && !state_complete(*merged_out)))
+    return GQA_ERR_INVALID_ARGUMENT;
+  if (!has_out_state && !out) return GQA_ERR_INVALID_ARGUMENT;
+  if (out && out_dtype != GQA_F32 && out_dtype != GQA_BF16) return GQA_ERR_SHAPE_MISMATCH;
+  if (static_cast<int64_t>(rows) * num_states * head_dim > (int64_t(1) << 40)) return GQA_ERR_INVALID_ARGUMENT;
+  // the merge kernel reads acc rows with 8- (D=64) or 16-byte (D=128) vector loads
+  if (num_states > 0 && (reinterpret_cast<uintptr_t>(states->acc) & 15u)) return GQA_ERR_SHAPE_MISMATCH;
+  const void* ptrs[] = {num_states > 0 ? states->m : nullptr, num_states > 0 ? states->l : nullptr,
+                        num_states > 0 ? states->acc : nullptr, has_carry ? carry_in->m : nullptr,
+                        has_carry ? carry_in->l : nullptr, has_carry ? carry_in->acc : nullptr,
+                        has_out_state ? merged_out->m : nullptr, has_out_state ? merged_out->l : nullptr,
+                        has_out_state ? merged_out->acc : nullptr, out};
+  for (const void* q : ptrs)
+    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
+  if (has_out_state && num_states > 0 &&
+      (merged_out->m == states->m || merged_out->l == states->l || merged_out->acc == states->acc))
+    return GQA_ERR_INVALID_ARGUMENT;
+  if (rows == 0) return GQA_OK;
+  MergeArgs m;
+  m.m = num_states > 0 ? states->m : nullptr;
+  m.l = num_states > 0 ? states->l : nullptr;
+  m.acc = num_states > 0 ? states->acc : nullptr;
+  m.rows = rows;
+  m.S = num_states;
+  m.offsets = nullptr;
+  m.H = 1;
+  m.chunk_len = 1;
+  m.max_len = 0;
+  m.cm = has_carry ? carry_in->m : nullptr;
+  m.cl = has_carry ? carry_in->l : nullptr;
+  m.cacc = has_carry ? carry_in->acc : nullptr;
+  m.om = has_out_state ? merged_out->m : nullptr;
+  m.ol = has_out_state ? merged_out->l : nullptr;
+  m.oacc = has_out_state ? merged_out->acc : nullptr;
+  m.out = out;
+  m.out_bf16 = out_dtype == GQA_BF16 ? 1 : 0;
+  if (launch_merge_any(head_dim, m, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GQA_ERR_DEVICE;
+  return GQA_OK;
+}
+
+gqa_status gqa_softmax_merge(const gqa_state* states, int32_t rows, int32_t num_states, int32_t head_dim,
+                             const gqa_state* carry_in, const gqa_state* merged_out, void* out,
+                             int32_t out_dtype, gqa_stream_t stream) {
+  return merge_common(states, rows, num_states, head_dim, carry_in, merged_out, out, out_dtype, stream);
+}
+
+gqa_status gqa_state_finalize(const gqa_state* state, int32_t rows, int32_t head_dim, void* out,
+                              int32_t out_dtype, gqa_stream_t stream) {
+  if (!out || !state) return GQA_ERR_INVALID_ARGUMENT;
+  return merge_common(state, rows, 1, head_dim, nullptr, nullptr, out, out_dtype, stream);
+}
+
+gqa_status gqa_get_device_error(void* workspace, gqa_stream_t stream) {
+  if (!workspace) return GQA_ERR_WORKSPACE;
+  if (!is_device_ptr(workspace)) return GQA_ERR_DEVICE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof word, cs) != cudaSuccess || cudaStreamSynchronize(cs) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_DEVICE;
+    }
+  }
+  if (word & gqa::kErrBadOffsets) return GQA_ERR_BAD_OFFSETS;
+  if (word & gqa::kErrTimeout) return GQA_ERR_TIMEOUT;
+  return GQA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+/*
+ * gqa_decode.h -- C ABI of the B200 (sm_100a) grouped-query decode attention library.
+ *
+ * One query token per sequence attends over that sequence's cached keys. Each
+ * query head h scores every cached key of its KV group g = h / (H / G) at scale
+ * score_scale (1/sqrt(head_dim) when 0), folds it into a running maximum m, a
+ * partition l and a weighted value sum acc, and the output is acc / l.
+ *
+ * Sources (the math and the argument conventions follow these pages):
+ *   [attn.rs]   needle_core `attn.rs` (docs.rs needle-core 0.3.1 source):
+ *               `KvCache` -- keys/values [max_len, num_kv_heads, head_dim];
+ *               `self_attn_incremental` -- kv head of Q head hi is hi / kv_repeat,
+ *               scale head_dim^-0.5, score -> softmax -> weighted sum of V;
+ *               `cross_attn_incremental` -- the same decode over a fixed cache.
+ *   [usearch]   USearch Rust docs, "Linear algebra", § Attention and the API
+ *               tables: `attend` folds every scored key into each head's running
+ *               maximum, partition and weighted value sum; outputs are already
+ *               divided by the partition, in the queries' scalar type; a carry of
+ *               one `DenseSoftmaxState` per query row folds the call into another
+ *               over the same queries; `score_scale` zero derives 1/sqrt(d);
+ *               `head_count` zero means one; ragged runs use Apache Arrow offsets;
+ *               refusals are `Status::ShapeMismatch`, `Status::Device`,
+ *               `Status::InvalidArgument`.
+ *   [cortiq]    cortiq_engine `NystromState` (docs.rs): under GQA every Q head of
+ *               a group reads the same K/V rows, so they are stored and read once
+ *               per group.
+ *   [dsa]       metrale `glm5next_dsa_ref/mod.rs`, `pool_states`: a softmax with
+ *               no valid entry gives weight 0, not NaN.
+ *
+ * Conventions for every entry point:
+ *   - Every tensor pointer is CALLER-OWNED DEVICE memory (cudaMalloc or a
+ *     framework allocator). The library allocates nothing, never synchronises
+ *     (except gqa_get_device_error) and enqueues all work on the caller's stream.
+ *   - Errors found on the host are returned synchronously and nothing is
+ *     launched. A launch failure returns GQA_ERR_DEVICE.
+ *   - Device-side findings (bad offsets, a pipeline wait that gave up) set bits
+ *     in the error word at the head of the workspace; gqa_get_device_error reads
+ *     and clears it.
+ *   - Dtypes: q/K/V are (fp32, fp32) or (bf16, bf16); any other pair is
+ *     GQA_ERR_SHAPE_MISMATCH. Accumulation is fp32 in both cases.
+ *   - head_dim is 64 or 128; heads per KV head (H / G) is 1..16.
+ */
+#ifndef GQA_DECODE_H
+#define GQA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream). NULL is the legacy default stream. */
+typedef struct CUstream_st* gqa_stream_t;
+
+/* Status codes. Refusals mirror [usearch] Status::InvalidArgument,
+ * Status::ShapeMismatch and Status::Device. */
+typedef enum {
+  GQA_OK = 0,
+  GQA_ERR_INVALID_ARGUMENT = 1, /* a size, count or required pointer is wrong  */
+  GQA_ERR_SHAPE_MISMATCH = 2,   /* unsupported dtype pair or misaligned tensor */
+  GQA_ERR_DEVICE = 3,           /* pointer not device memory, no device, launch failure */
+  GQA_ERR_WORKSPACE = 4,        /* workspace missing or smaller than required  */
+  GQA_ERR_BAD_OFFSETS = 5,      /* device-detected: offsets not monotone / beyond max_len */
+  GQA_ERR_TIMEOUT = 6           /* device-detected: a pipeline wait gave up    */
+} gqa_status;
+
+typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
+
+/* An online-softmax state per query row, structure of arrays, fp32 device memory:
+ *   m   [rows]        running maximum of the logits scale*q.k, natural-log units
+ *                     ([usearch] DenseSoftmaxState::maximum_score)
+ *   l   [rows]        partition: sum of e^{logit - m}  ([usearch] ::partition)
+ *   acc [rows, D]     unnormalised weighted value sum, sum e^{logit - m} v
+ * The output of a state is acc / l. A state with l == 0 is EMPTY whatever its m
+ * (identity of the merge); the library writes empty states as (-inf, 0, 0).
+ * A gqa_state with all three pointers NULL means "absent". */
+typedef struct {
+  float* m;
+  float* l;
+  float* acc;
+} gqa_state;
+
+/* Arguments of gqa_decode_attend. Set struct_size = sizeof(gqa_decode_params). */
+typedef struct {
+  uint32_t struct_size;
+  /* q [batch, num_heads, head_dim]; row b*H + h is head h of sequence b ([usearch]
+   * "row t * head_count + h of the queries is head h of token t"). */
+  const void* q;
+  int32_t q_dtype;           /* gqa_dtype */
+  /* K and V caches [max_len, num_kv_heads, head_dim], row stride
+   * num_kv_heads*head_dim ([attn.rs] KvCache). 16-byte aligned. */
+  const void* k;
+  const void* v;
+  int32_t kv_dtype;          /* gqa_dtype */
+  /* Arrow offsets [batch + 1], device int32: sequence b owns cache rows
+   * offsets[b] .. offsets[b+1]-1. Must satisfy 0 <= offsets[b] <= offsets[b+1]
+   * <= max_len; a violating sequence is treated as empty and flags
+   * GQA_ERR_BAD_OFFSETS in the device error word. */
+  const int32_t* offsets;
+  int32_t batch;             /* B >= 0; 0 is a no-op */
+  int32_t max_len;           /* rows allocated in the K/V caches (>= offsets[B]) */
+  int32_t max_seq_len;       /* host hint: longest sequence; 0 => max_len. A hint
+                                that is too small stays correct, only slower. */
+  int32_t num_heads;         /* H >= 1 */
+  int32_t num_kv_heads;      /* G; 0 => G = H. H % G must be 0, H / G <= 16 */
+  int32_t head_dim;          /* D: 64 or 128 */
+  float score_scale;         /* logit scale; 0 => 1/sqrt(head_dim); finite */
+  /* Optional carry, one state per query row [B*H], folded into this call
+   * ([usearch] DenseAttendConfig::carry). All-NULL = no carry. */
+  gqa_state carry_in;
+  /* Optional merged state out [B*H]; may alias carry_in exactly. */
+  gqa_state state_out;
+  /* Optional output [B, H, D] in out_dtype (acc / l, rounded to nearest even
+   * for bf16; 0 for a row with no keys and no carry). */
+  void* out;
+  int32_t out_dtype;         /* gqa_dtype; conventionally q_dtype */
+  /* Optional raw per-split states [B*H, num_splits] (m, l) and
+   * [B*H, num_splits, D] (acc): split s of a sequence covers its keys
+   * [s*chunk_len, (s+1)*chunk_len) (the last split also takes any remainder).
+   * Splits with no keys are written as empty states. The carry is NOT folded
+   * into these; merge them with gqa_softmax_merge. */
+  gqa_state partials_out;
+  int32_t num_splits;        /* 0 => chosen by the library's heuristic */
+  /* Scratch: at least gqa_decode_workspace_size() bytes, 256-byte aligned,
+   * initialised once with gqa_workspace_init. Not shared by calls that overlap. */
+  void* workspace;
+  size_t workspace_bytes;
+} gqa_decode_params;
+
+/* Bytes of workspace gqa_decode_attend needs for these params, and the
+ * split plan it will use (either may be NULL). Host only; reads the current
+ * device's SM count. At least out, state_out or partials_out must be set. */
+gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes,
+                                     int32_t* num_splits, int32_t* chunk_len);
+
+/* Zero the workspace's error word. Call once after allocating a workspace. */
+gqa_status gqa_workspace_init(void* workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/* Decode attention with a mergeable online-softmax state ([attn.rs]
+ * self_attn_incremental / cross_attn_incremental without the projections;
+ * [usearch] § Attention with its carry). Launches the split-KV partition kernel
+ * and, when out or state_out is requested, the merge/finalize kernel, on
+ * `stream`. Asynchronous. */
+gqa_status gqa_decode_attend(const gqa_decode_params* params, gqa_stream_t stream);
+
+/* Merge num_states states per row ([usearch] carry: partial-softmax rescaling):
+ *   M = max m_i,  L = sum l_i e^{m_i - M},  ACC = sum acc_i e^{m_i - M}
+ * over the non-empty states (l_i != 0) of each row, plus carry_in when given.
+ *   states      m, l [rows, num_states], acc [rows, num_states, head_dim]
+ *   carry_in    NULL or a state [rows]
+ *   merged_out  NULL or a state [rows]; may alias carry_in, not states
+ *   out         NULL or [rows, head_dim] in out_dtype: ACC / L (0 when L == 0)
+ * At least one of merged_out / out must be given. rows may be 0. */
+gqa_status gqa_softmax_merge(const gqa_state* states, int32_t rows, int32_t num_states,
+                             int32_t head_dim, const gqa_state* carry_in,
+                             const gqa_state* merged_out, void* out, int32_t out_dtype,
+                             gqa_stream_t stream);
+
+/* out = acc / l per row (0 when l == 0), cast to out_dtype ([usearch]: outputs
+ * land already divided by the partition). state [rows], out [rows, head_dim]. */
+gqa_status gqa_state_finalize(const gqa_state* state, int32_t rows, int32_t head_dim, void* out,
+                              int32_t out_dtype, gqa_stream_t stream);
+
+/* Synchronise `stream`, read and clear the workspace's device error word.
+ * Returns GQA_OK, GQA_ERR_BAD_OFFSETS or GQA_ERR_TIMEOUT (the first set). */
+gqa_status gqa_get_device_error(void* workspace, gqa_stream_t stream);
+
+/* The split plan of the heuristic, exposed for inspection and tests (host only):
+ * chunk_len is a multiple of 64 and num_splits = ceil(max_seq_len / chunk_len).
+ * total_rows is the expected sum of sequence lengths (<= batch*max_seq_len);
+ * resident_ctas is the number of partition CTAs the GPU holds at once. */
+gqa_status gqa_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
+                           int64_t total_rows, int32_t resident_ctas, int32_t* chunk_len,
+                           int32_t* num_splits);
+
+/* Human-readable name of a status. Never NULL. */
+const char* gqa_status_string(gqa_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_DECODE_H */
