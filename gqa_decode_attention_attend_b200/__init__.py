@@ -352,3 +352,32 @@ def gqa_plan_splits(batch, num_kv_heads, max_seq_len, total_rows, resident_ctas)
 
 def default_scale(head_dim):
     return 1.0 / math.sqrt(head_dim)
+
+
+def gqa_decode_attend_static_workspace(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scale=0.0,
+                                       carry=None, state_out=None, out=None, out_dtype=None,
+                                       partials_out=None, want_out=None, num_splits=0, max_seq_len=0,
+                                       max_len=None, stream=None):
+    """gqa_decode_attend for callers that cannot provide scratch memory.
+
+    Same arguments and result as gqa_decode_attend minus the workspace: the
+    library keeps its scratch in a fixed 16 MiB device array of its own (see
+    include/gqa_decode.h for who needs this and its limits). Calls that may run
+    concurrently on the GPU share that array and must be serialised.
+    """
+    torch = _torch()
+    lib = load_library()
+    fn = lib.gqa_decode_attend_static_workspace
+    fn.argtypes = [ctypes.POINTER(_CParams), ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    if want_out is None:
+        want_out = out is not None or (state_out is None and partials_out is None)
+    odt = _dtype_code(q) if out_dtype is None else _dtype_code(torch.empty(0, dtype=out_dtype))
+    if want_out and out is None:
+        out = torch.empty(q.shape, dtype=_torch_dtype(odt), device=q.device)
+    if out is not None:
+        odt = _dtype_code(out)
+    p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
+                partials_out, num_splits, max_seq_len, max_len)
+    _check(fn(ctypes.byref(p), _stream_handle(stream)), "gqa_decode_attend_static_workspace")
+    return out

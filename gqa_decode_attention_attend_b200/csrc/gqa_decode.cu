@@ -516,3 +516,132 @@ gqa_status gqa_get_device_error(void* workspace, gqa_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ============================================================================
+// Decode attention without a caller-supplied workspace.
+//
+// Some callers cannot hand the library scratch memory: code that runs where a
+// device allocation is not allowed or not safe (a plugin inside a host engine
+// that owns every device buffer and offers no workspace, a fixed-budget or
+// real-time deployment that forbids allocation after start-up, or a callback
+// in which cudaMalloc would implicitly synchronise the device). For them the
+// scratch of gqa_decode_attend (the error word and the per-split partial
+// states) lives in the file-scope device array below, which the CUDA module
+// loader sets aside, zero-filled, on every GPU that loads this library and
+// keeps until the process exits.
+// ============================================================================
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB per GPU
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device. The host-side
+// symbol is only a stand-in, so the address is looked up once per device
+// (with that device current) and cached.
+void* static_scratch_address(int dev) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_static_scratch_addr[dev] = p;
+  }
+  return g_static_scratch_addr[dev];
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_decode_attend_static_workspace(const gqa_decode_params* p,
+                                                         gqa_stream_t stream) {
+  Resolved r;
+  gqa_status st = resolve(p, &r, true);
+  if (st != GQA_OK) return st;
+  if (r.bytes > kStaticScratchBytes) return GQA_ERR_WORKSPACE;   // scratch need above the array
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(static_scratch_address(dev));
+  if (ws == nullptr) return GQA_ERR_DEVICE;
+  const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out,
+                        p->carry_in.m, p->carry_in.l, p->carry_in.acc,
+                        p->state_out.m, p->state_out.l, p->state_out.acc,
+                        p->partials_out.m, p->partials_out.l, p->partials_out.acc};
+  for (const void* q : ptrs)
+    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
+  if (r.B == 0) return GQA_OK;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  // The array keeps whatever the previous call left in it. Only the error word
+  // must start at zero (the partial states are written before they are read).
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), cs) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  PartitionArgs a;
+  a.q = p->q;
+  a.k = p->k;
+  a.v = p->v;
+  a.offsets = p->offsets;
+  a.B = r.B;
+  a.H = r.H;
+  a.G = r.G;
+  a.hpk = r.hpk;
+  a.max_len = r.max_len;
+  a.chunk_len = r.chunk;
+  a.num_splits = r.S;
+  a.scale_log2 = r.scale * gqa::kLog2e;
+  if (r.has_partials) {
+    a.part_m = p->partials_out.m;
+    a.part_l = p->partials_out.l;
+    a.part_acc = p->partials_out.acc;
+    a.write_empty = 1;
+  } else {
+    a.part_m = reinterpret_cast<float*>(ws + r.off_m);
+    a.part_l = reinterpret_cast<float*>(ws + r.off_l);
+    a.part_acc = reinterpret_cast<float*>(ws + r.off_acc);
+    a.write_empty = 0;
+  }
+  a.err = reinterpret_cast<uint32_t*>(ws);
+
+  if (r.max_len > 0 || r.has_partials) {
+    CUtensorMap tk, tv;
+    const int map_rows = r.max_len > 0 ? r.max_len : 1;
+    const void* kb = r.max_len > 0 ? p->k : static_cast<const void*>(ws);
+    const void* vb = r.max_len > 0 ? p->v : static_cast<const void*>(ws);
+    if (r.bf16 && (!make_kv_map(&tk, kb, map_rows, r.G, r.D) || !make_kv_map(&tv, vb, map_rows, r.G, r.D)))
+      return GQA_ERR_DEVICE;
+    if (launch_partition(r, a, &tk, &tv, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+  }
+  if (r.want_merge) {
+    MergeArgs m;
+    m.m = a.part_m;
+    m.l = a.part_l;
+    m.acc = a.part_acc;
+    m.rows = r.B * r.H;
+    m.S = r.S;
+    m.offsets = p->offsets;
+    m.H = r.H;
+    m.chunk_len = r.chunk;
+    m.max_len = r.max_len;
+    const bool has_carry = state_present(p->carry_in);
+    m.cm = has_carry ? p->carry_in.m : nullptr;
+    m.cl = has_carry ? p->carry_in.l : nullptr;
+    m.cacc = has_carry ? p->carry_in.acc : nullptr;
+    const bool has_so = state_present(p->state_out);
+    m.om = has_so ? p->state_out.m : nullptr;
+    m.ol = has_so ? p->state_out.l : nullptr;
+    m.oacc = has_so ? p->state_out.acc : nullptr;
+    m.out = p->out;
+    m.out_bf16 = r.out_bf16;
+    if (launch_merge_any(r.D, m, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+  }
+  return GQA_OK;
+}

@@ -144,6 +144,34 @@ gqa_status gqa_workspace_init(void* workspace, size_t workspace_bytes, gqa_strea
  * `stream`. Asynchronous. */
 gqa_status gqa_decode_attend(const gqa_decode_params* params, gqa_stream_t stream);
 
+/* Decode attention exactly as gqa_decode_attend, for callers that cannot
+ * provide scratch memory. The pages this library follows have no counterpart
+ * of this entry point; it exists for deployment reasons only.
+ *
+ * Who needs it: code that must not allocate device memory or cannot obtain it
+ * -- a plugin living inside a host engine that owns every device buffer and
+ * gives the plugin no workspace, a fixed-budget or real-time service that
+ * forbids allocations after start-up, or a callback in which cudaMalloc would
+ * synchronise the device.
+ *
+ * params->workspace and params->workspace_bytes are ignored; every other field
+ * means what it means for gqa_decode_attend, and the caller still passes all
+ * inputs and outputs. The scratch is a 16 MiB device array inside the library
+ * (the CUDA loader reserves it on every GPU that loads the library, until the
+ * process exits). The call allocates nothing itself.
+ *   - A call whose scratch need (gqa_decode_workspace_size) exceeds 16 MiB is
+ *     refused with GQA_ERR_WORKSPACE.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     calls that may run at the same time on the GPU (different streams, or
+ *     different host threads) race on it and must be serialised by the caller.
+ *   - The device error word is cleared at the start of each call and is not
+ *     readable through gqa_get_device_error; use gqa_decode_attend with a
+ *     workspace to diagnose malformed offsets. */
+gqa_status gqa_decode_attend_static_workspace(const gqa_decode_params* params, gqa_stream_t stream);
+
 /* Merge num_states states per row ([usearch] carry: partial-softmax rescaling):
  *   M = max m_i,  L = sum l_i e^{m_i - M},  ACC = sum acc_i e^{m_i - M}
  * over the non-empty states (l_i != 0) of each row, plus carry_in when given.
