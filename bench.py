@@ -1,8 +1,9 @@
 #!/usr/bin/env python
 """Benchmark of the decode-attention hot path on B200.
 
-One step = one gqa_decode_attend call over the whole batch (split-KV partition
-kernel + merge/finalize kernel) on the 16-sequence bf16 workload: batch 16,
+One step = one gqa_decode_attend call over the whole batch (one launch of the
+split-KV partition kernel, whose last CTA per sequence and KV head merges the
+splits and writes the output) on the 16-sequence bf16 workload: batch 16,
 32 Q / 8 KV heads, head_dim 128, 4096 cached keys per sequence, q/K/V iid
 N(0,1), bf16 output. Inputs are resident in HBM before the timed region; two
 copies of the 256 MiB cache are alternated so consecutive steps never read a
@@ -48,6 +49,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--quick", action="store_true",
+                    help="timed loop and kernel timing only (no clock sampling, e2e or CPU "
+                         "baseline); for profiler launch lists")
     return ap.parse_args()
 
 
@@ -218,7 +222,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert gqa.gqa_get_device_error(ws) == 0
 
-    sampler = ClockSampler(local) if rank == 0 or world > 1 else None
+    sampler = ClockSampler(local) if not args.quick else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
@@ -235,7 +239,7 @@ def run_ours(args):
     # keep the same load for at least ~1.5 s so the clock sampler sees it
     extra_t0 = time.perf_counter()
     i = 0
-    while ms_total / 1e3 + (time.perf_counter() - extra_t0) < 1.5:
+    while sampler and ms_total / 1e3 + (time.perf_counter() - extra_t0) < 1.5:
         for _ in range(200):
             step(i)
             i += 1
@@ -262,7 +266,7 @@ def run_ours(args):
 
     for i in range(5):
         part_only(i)
-    n_part = max(args.steps, 50)
+    n_part = args.steps if args.quick else max(args.steps, 50)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -293,24 +297,25 @@ def run_ours(args):
                               max_seq_len=w.max_seq_len, workspace=ws, stream=stream)
         hout.copy_(out, non_blocking=True)
 
-    for _ in range(2):
+    n_e2e = 0 if args.quick else args.e2e_steps
+    for _ in range(2 if n_e2e else 0):
         e2e_step()
     torch.cuda.synchronize()
     barrier()
     x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     x0.record(stream)
-    for _ in range(args.e2e_steps):
+    for _ in range(n_e2e):
         e2e_step()
     x1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([x0.elapsed_time(x1) / args.e2e_steps], dtype=torch.float64, device=dev)
+    te = torch.tensor([x0.elapsed_time(x1) / max(n_e2e, 1)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_ms = float(te.item())
     e2e_value = kv_bytes * world / (e2e_ms / 1e3) / 1e9
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
         gbs, qh, cores, sample = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
                "queries_heads_per_s": qh}
@@ -349,7 +354,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -96,7 +96,7 @@ def load_library(path=None):
     lib.gqa_softmax_merge.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
     lib.gqa_state_finalize.argtypes = [ps, i32, i32, sp, i32, sp]
     lib.gqa_get_device_error.argtypes = [sp, sp]
-    lib.gqa_plan_splits.argtypes = [i32, i32, i32, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.gqa_plan_splits.argtypes = [i32, i32, i32, i64, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.gqa_status_string.argtypes = [ctypes.c_int]
     lib.gqa_status_string.restype = ctypes.c_char_p
     lib.gqa_version.argtypes = []
@@ -340,13 +340,13 @@ def gqa_workspace_init(workspace, stream=None):
                                              _stream_handle(stream)), "gqa_workspace_init")
 
 
-def gqa_plan_splits(batch, num_kv_heads, max_seq_len, total_rows, resident_ctas):
+def gqa_plan_splits(batch, num_kv_heads, max_seq_len, total_rows, sm_count=148, ctas_per_sm=2):
     """(chunk_len, num_splits) of the library's split heuristic (host only)."""
     c = ctypes.c_int32()
     s = ctypes.c_int32()
     _check(load_library().gqa_plan_splits(int(batch), int(num_kv_heads), int(max_seq_len),
-                                          int(total_rows), int(resident_ctas), ctypes.byref(c),
-                                          ctypes.byref(s)), "gqa_plan_splits")
+                                          int(total_rows), int(sm_count), int(ctas_per_sm),
+                                          ctypes.byref(c), ctypes.byref(s)), "gqa_plan_splits")
     return c.value, s.value
 
 

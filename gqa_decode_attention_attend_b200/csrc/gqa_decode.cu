@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -19,6 +20,11 @@ using gqa::PartitionArgs;
 
 constexpr int kVersion = 100;          // 0.1.0
 constexpr size_t kHeaderBytes = 256;   // error word + reserved
+// Merge tickets live in a fixed region right after the header that nothing else
+// ever uses, so the zeros left by gqa_workspace_init and by every completed call
+// survive calls of any shape. Batches with more (sequence, KV head) segments
+// than it holds get a region after the partial states, cleared on each call.
+constexpr size_t kTicketSlots = 65536;
 constexpr int kChunkQuantum = 64;      // rows per pipeline stage of the bf16 kernel
 constexpr int kMaxHeadsPerKv = 16;
 constexpr int kMaxDevices = 64;
@@ -145,41 +151,78 @@ struct Resolved {
   bool want_merge;      // out or state_out requested
   bool has_partials;    // caller's partials_out
   int S, chunk;         // split plan
-  int resident;         // partition CTAs resident on the whole GPU
+  int sm_count;         // SMs of the device (0 when not queried)
+  int per_sm;           // partition CTAs resident per SM
   size_t bytes;         // workspace bytes
-  size_t off_m, off_l, off_acc;
+  size_t off_m, off_l, off_acc, off_counters;
+  bool clear_counters;  // counters outside the fixed ticket region
 };
 
 int nt_of(int hpk) { return hpk <= 8 ? 1 : 2; }
 
+// Split heuristic. A split is a chunk of chunk_len keys (a multiple of the
+// 64-row pipeline stage) of one sequence; one CTA owns one (sequence, KV head,
+// split) tile, so a call launches batch * num_kv_heads * num_splits CTAs.
+//
+// Equal-length batch: the kernel is HBM-bound as soon as about one CTA per SM
+// is streaming, and every CTA does the same work, so the time is set by how
+// the CTAs fill the `resident` slots. A last partial wave costs as much as
+// max(its CTAs, sm_count) CTAs would (each CTA's own stream is bounded). The
+// plan minimises
+//     waves * (chunk_len + 128) + 4 * num_splits
+// (128 rows ~ a CTA's fixed prologue/epilogue, 4 rows ~ one more partial state
+// in the merge), ties going to fewer splits.
+// Ragged batch (total_rows below batch * max_seq_len): the tiles are uneven, so
+// the plan aims at ~8 waves of CTAs and lets the block scheduler balance them.
 gqa_status plan_impl(int32_t batch, int32_t G, int32_t max_seq_len, int64_t total_rows,
-                     int32_t resident, int32_t* chunk_len, int32_t* num_splits) {
-  if (batch < 0 || G <= 0 || max_seq_len < 0 || resident <= 0 || !chunk_len || !num_splits)
+                     int32_t sm_count, int32_t ctas_per_sm, int32_t* chunk_len, int32_t* num_splits) {
+  if (batch < 0 || G <= 0 || max_seq_len < 0 || sm_count <= 0 || ctas_per_sm <= 0 || !chunk_len ||
+      !num_splits)
     return GQA_ERR_INVALID_ARGUMENT;
+  const int64_t q = kChunkQuantum;
   if (max_seq_len == 0 || batch == 0) {
     *chunk_len = kChunkQuantum;
     *num_splits = 1;
     return GQA_OK;
   }
-  const int64_t full = static_cast<int64_t>(batch) * max_seq_len;
+  const int64_t resident = static_cast<int64_t>(sm_count) * ctas_per_sm;
+  const int64_t N = max_seq_len;
+  const int64_t full = static_cast<int64_t>(batch) * N;
   if (total_rows <= 0 || total_rows > full) total_rows = full;
-  const bool uniform = total_rows == full;
-  // Target enough CTAs that every SM holds several from the start and the last
-  // ones are short: 2 x resident for equal-length sequences, 8 x resident for a
-  // ragged batch (where chunk lengths vary).
-  const int64_t target = static_cast<int64_t>(resident) * (uniform ? 2 : 8);
-  const int64_t units = total_rows * G;                          // (row, KV head) pairs
-  int64_t chunk = (units + target - 1) / target;
-  const int64_t cap = (static_cast<int64_t>(max_seq_len) + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum;
-  chunk = (chunk + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum;
-  if (chunk < 4 * kChunkQuantum) chunk = 4 * kChunkQuantum;      // amortise the per-CTA prologue
-  if (chunk > cap) chunk = cap;
-  int64_t splits = (max_seq_len + chunk - 1) / chunk;
-  // even out the splits of a full-length sequence
-  chunk = ((max_seq_len + splits - 1) / splits + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum;
-  splits = (max_seq_len + chunk - 1) / chunk;
-  *chunk_len = static_cast<int32_t>(chunk);
-  *num_splits = static_cast<int32_t>(splits);
+  const int64_t max_splits = (N + q - 1) / q;
+  if (total_rows < full) {
+    const int64_t target = resident * 8;
+    int64_t chunk = (total_rows * G + target - 1) / target;
+    chunk = (chunk + q - 1) / q * q;
+    if (chunk < 4 * q) chunk = 4 * q;
+    if (chunk > max_splits * q) chunk = max_splits * q;
+    int64_t splits = (N + chunk - 1) / chunk;
+    chunk = ((N + splits - 1) / splits + q - 1) / q * q;
+    *chunk_len = static_cast<int32_t>(chunk);
+    *num_splits = static_cast<int32_t>((N + chunk - 1) / chunk);
+    return GQA_OK;
+  }
+  const int64_t segs = static_cast<int64_t>(batch) * G;
+  double best = 0.0;
+  int64_t best_chunk = 0, best_splits = 0;
+  const int64_t limit = std::min<int64_t>(max_splits, 4 * resident / segs + 2);
+  for (int64_t S = 1; S <= limit; ++S) {
+    const int64_t chunk = ((N + S - 1) / S + q - 1) / q * q;
+    const int64_t splits = (N + chunk - 1) / chunk;
+    if (splits != S) continue;                      // same plan as a smaller S
+    const int64_t ctas = segs * S;
+    const int64_t rem = ctas % resident;
+    const double waves = static_cast<double>(ctas / resident) +
+                         (rem ? static_cast<double>(std::max<int64_t>(rem, sm_count)) / resident : 0.0);
+    const double cost = waves * static_cast<double>(chunk + 128) + 4.0 * S;
+    if (best_splits == 0 || cost < best) {
+      best = cost;
+      best_chunk = chunk;
+      best_splits = S;
+    }
+  }
+  *chunk_len = static_cast<int32_t>(best_chunk);
+  *num_splits = static_cast<int32_t>(best_splits);
   return GQA_OK;
 }
 
@@ -217,21 +260,28 @@ gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
   if (p->out && p->out_dtype != GQA_F32 && p->out_dtype != GQA_BF16) return GQA_ERR_SHAPE_MISMATCH;
   r->bf16 = p->kv_dtype == GQA_BF16;
   r->out_bf16 = p->out_dtype == GQA_BF16 ? 1 : 0;
-  const uintptr_t align_or = reinterpret_cast<uintptr_t>(p->q) | reinterpret_cast<uintptr_t>(p->k) |
-                             reinterpret_cast<uintptr_t>(p->v);
+  // q/K/V feed 32-bit and TMA loads; out and every acc array are read and
+  // written four floats (or four bf16) at a time.
+  const uintptr_t align_or =
+      reinterpret_cast<uintptr_t>(p->q) | reinterpret_cast<uintptr_t>(p->k) |
+      reinterpret_cast<uintptr_t>(p->v) | reinterpret_cast<uintptr_t>(p->out) |
+      reinterpret_cast<uintptr_t>(p->carry_in.acc) | reinterpret_cast<uintptr_t>(p->state_out.acc) |
+      reinterpret_cast<uintptr_t>(p->partials_out.acc);
   if (align_or & 15u) return GQA_ERR_SHAPE_MISMATCH;
   if (!std::isfinite(p->score_scale)) return GQA_ERR_INVALID_ARGUMENT;
   r->scale = p->score_scale != 0.f ? p->score_scale : 1.0f / sqrtf(static_cast<float>(r->D));
   if (static_cast<int64_t>(r->B) * r->H * r->D > INT32_MAX) return GQA_ERR_INVALID_ARGUMENT;
 
-  r->resident = 0;
+  r->sm_count = 148;     // B200; replaced by the device's own count below
+  r->per_sm = 2;
   if (need_device) {
     int dev;
     const DeviceInfo* di = device_info(&dev);
     if (!di) return GQA_ERR_DEVICE;
     const int per_sm = r->bf16 ? di->resident_bf16[r->D == 128][nt_of(r->hpk) - 1]
                                : di->resident_f32[r->D == 128];
-    r->resident = di->sm_count * (per_sm > 0 ? per_sm : 1);
+    r->sm_count = di->sm_count;
+    r->per_sm = per_sm > 0 ? per_sm : 1;
   }
   // split plan
   if (p->num_splits > 0) {
@@ -241,8 +291,7 @@ gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
     r->chunk = static_cast<int>(chunk);
   } else {
     int32_t c, s;
-    const int64_t rows_hint = r->max_len;
-    gqa_status st = plan_impl(r->B, r->G, r->max_seq_len, rows_hint, r->resident > 0 ? r->resident : 296, &c, &s);
+    gqa_status st = plan_impl(r->B, r->G, r->max_seq_len, r->max_len, r->sm_count, r->per_sm, &c, &s);
     if (st != GQA_OK) return st;
     r->S = s;
     r->chunk = c;
@@ -250,7 +299,13 @@ gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
   if (static_cast<int64_t>(r->B) * r->S * r->G > INT32_MAX) return GQA_ERR_INVALID_ARGUMENT;
   // workspace: header, then internal partial states when merging without the caller's
   r->bytes = kHeaderBytes;
-  r->off_m = r->off_l = r->off_acc = 0;
+  r->off_m = r->off_l = r->off_acc = r->off_counters = 0;
+  r->clear_counters = false;
+  const size_t segs = static_cast<size_t>(r->B) * r->G;
+  if (r->want_merge) {
+    r->off_counters = r->bytes;
+    r->bytes += kTicketSlots * sizeof(uint32_t);
+  }
   if (r->want_merge && !r->has_partials) {
     const size_t n = static_cast<size_t>(r->B) * r->H * r->S;
     r->off_m = r->bytes;
@@ -259,6 +314,11 @@ gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
     r->bytes += align256(n * sizeof(float));
     r->off_acc = r->bytes;
     r->bytes += align256(n * r->D * sizeof(float));
+  }
+  if (r->want_merge && segs > kTicketSlots) {
+    r->off_counters = r->bytes;
+    r->bytes += align256(segs * sizeof(uint32_t));
+    r->clear_counters = true;
   }
   return GQA_OK;
 }
@@ -308,58 +368,10 @@ cudaError_t launch_partition(const Resolved& r, const PartitionArgs& a, const CU
   return launch_f32<64, 16>(a, grid, st);
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* gqa_status_string(gqa_status s) {
-  switch (s) {
-    case GQA_OK: return "GQA_OK";
-    case GQA_ERR_INVALID_ARGUMENT: return "GQA_ERR_INVALID_ARGUMENT";
-    case GQA_ERR_SHAPE_MISMATCH: return "GQA_ERR_SHAPE_MISMATCH";
-    case GQA_ERR_DEVICE: return "GQA_ERR_DEVICE";
-    case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE";
-    case GQA_ERR_BAD_OFFSETS: return "GQA_ERR_BAD_OFFSETS";
-    case GQA_ERR_TIMEOUT: return "GQA_ERR_TIMEOUT";
-  }
-  return "GQA_ERR_UNKNOWN";
-}
-
-int32_t gqa_version(void) { return kVersion; }
-
-gqa_status gqa_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len, int64_t total_rows,
-                           int32_t resident_ctas, int32_t* chunk_len, int32_t* num_splits) {
-  return plan_impl(batch, num_kv_heads, max_seq_len, total_rows, resident_ctas, chunk_len, num_splits);
-}
-
-gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes, int32_t* num_splits,
-                                     int32_t* chunk_len) {
-  Resolved r;
-  gqa_status st = resolve(params, &r, true);
-  if (st != GQA_OK) return st;
-  if (bytes) *bytes = r.bytes;
-  if (num_splits) *num_splits = r.S;
-  if (chunk_len) *chunk_len = r.chunk;
-  return GQA_OK;
-}
-
-gqa_status gqa_workspace_init(void* workspace, size_t workspace_bytes, gqa_stream_t stream) {
-  if (!workspace || workspace_bytes < kHeaderBytes) return GQA_ERR_WORKSPACE;
-  if (!is_device_ptr(workspace)) return GQA_ERR_DEVICE;
-  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
-    cudaGetLastError();
-    return GQA_ERR_DEVICE;
-  }
-  return GQA_OK;
-}
-
-gqa_status gqa_decode_attend(const gqa_decode_params* p, gqa_stream_t stream) {
-  Resolved r;
-  gqa_status st = resolve(p, &r, true);
-  if (st != GQA_OK) return st;
-  if (!p->workspace || p->workspace_bytes < r.bytes) return GQA_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
-  const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out, p->workspace,
+// Pointer checks and the single launch of a decode call, with the scratch at `ws`
+// (the caller's workspace, or the library's static array).
+gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* ws, cudaStream_t cs) {
+  const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out,
                         p->carry_in.m, p->carry_in.l, p->carry_in.acc,
                         p->state_out.m, p->state_out.l, p->state_out.acc,
                         p->partials_out.m, p->partials_out.l, p->partials_out.acc};
@@ -367,8 +379,6 @@ gqa_status gqa_decode_attend(const gqa_decode_params* p, gqa_stream_t stream) {
     if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
   if (r.B == 0) return GQA_OK;
 
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
   PartitionArgs a;
   a.q = p->q;
   a.k = p->k;
@@ -394,44 +404,91 @@ gqa_status gqa_decode_attend(const gqa_decode_params* p, gqa_stream_t stream) {
     a.write_empty = 0;
   }
   a.err = reinterpret_cast<uint32_t*>(ws);
+  a.merge = r.want_merge ? 1 : 0;
+  a.counters = r.want_merge ? reinterpret_cast<uint32_t*>(ws + r.off_counters) : nullptr;
+  const bool has_carry = state_present(p->carry_in);
+  a.cm = has_carry ? p->carry_in.m : nullptr;
+  a.cl = has_carry ? p->carry_in.l : nullptr;
+  a.cacc = has_carry ? p->carry_in.acc : nullptr;
+  const bool has_so = state_present(p->state_out);
+  a.om = has_so ? p->state_out.m : nullptr;
+  a.ol = has_so ? p->state_out.l : nullptr;
+  a.oacc = has_so ? p->state_out.acc : nullptr;
+  a.out = p->out;
+  a.out_bf16 = r.out_bf16;
 
-  if (r.max_len > 0 || r.has_partials) {
-    // With no cache rows every tile is empty and no load is issued, but a
-    // tensor map still needs a non-zero extent and a valid aligned base: the
-    // workspace stands in for the (possibly null) empty caches.
-    CUtensorMap tk, tv;
-    const int map_rows = r.max_len > 0 ? r.max_len : 1;
-    const void* kb = r.max_len > 0 ? p->k : p->workspace;
-    const void* vb = r.max_len > 0 ? p->v : p->workspace;
-    if (r.bf16 && (!make_kv_map(&tk, kb, map_rows, r.G, r.D) || !make_kv_map(&tv, vb, map_rows, r.G, r.D)))
-      return GQA_ERR_DEVICE;
-    if (launch_partition(r, a, &tk, &tv, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+  // With no cache rows every tile is empty and no load is issued, but a tensor
+  // map still needs a non-zero extent and a valid aligned base: the scratch
+  // stands in for the (possibly null) empty caches.
+  CUtensorMap tk, tv;
+  const int map_rows = r.max_len > 0 ? r.max_len : 1;
+  const void* kb = r.max_len > 0 ? p->k : static_cast<const void*>(ws);
+  const void* vb = r.max_len > 0 ? p->v : static_cast<const void*>(ws);
+  if (r.bf16 && (!make_kv_map(&tk, kb, map_rows, r.G, r.D) || !make_kv_map(&tv, vb, map_rows, r.G, r.D)))
+    return GQA_ERR_DEVICE;
+  if (r.clear_counters &&
+      cudaMemsetAsync(a.counters, 0, static_cast<size_t>(r.B) * r.G * sizeof(uint32_t), cs) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
   }
+  if (launch_partition(r, a, &tk, &tv, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+  return GQA_OK;
+}
 
-  if (r.want_merge) {
-    MergeArgs m;
-    m.m = a.part_m;
-    m.l = a.part_l;
-    m.acc = a.part_acc;
-    m.rows = r.B * r.H;
-    m.S = r.S;
-    m.offsets = p->offsets;
-    m.H = r.H;
-    m.chunk_len = r.chunk;
-    m.max_len = r.max_len;
-    const bool has_carry = state_present(p->carry_in);
-    m.cm = has_carry ? p->carry_in.m : nullptr;
-    m.cl = has_carry ? p->carry_in.l : nullptr;
-    m.cacc = has_carry ? p->carry_in.acc : nullptr;
-    const bool has_so = state_present(p->state_out);
-    m.om = has_so ? p->state_out.m : nullptr;
-    m.ol = has_so ? p->state_out.l : nullptr;
-    m.oacc = has_so ? p->state_out.acc : nullptr;
-    m.out = p->out;
-    m.out_bf16 = r.out_bf16;
-    if (launch_merge_any(r.D, m, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+}  // namespace
+
+extern "C" {
+
+const char* gqa_status_string(gqa_status s) {
+  switch (s) {
+    case GQA_OK: return "GQA_OK";
+    case GQA_ERR_INVALID_ARGUMENT: return "GQA_ERR_INVALID_ARGUMENT";
+    case GQA_ERR_SHAPE_MISMATCH: return "GQA_ERR_SHAPE_MISMATCH";
+    case GQA_ERR_DEVICE: return "GQA_ERR_DEVICE";
+    case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE";
+    case GQA_ERR_BAD_OFFSETS: return "GQA_ERR_BAD_OFFSETS";
+    case GQA_ERR_TIMEOUT: return "GQA_ERR_TIMEOUT";
+  }
+  return "GQA_ERR_UNKNOWN";
+}
+
+int32_t gqa_version(void) { return kVersion; }
+
+gqa_status gqa_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len, int64_t total_rows,
+                           int32_t sm_count, int32_t ctas_per_sm, int32_t* chunk_len, int32_t* num_splits) {
+  return plan_impl(batch, num_kv_heads, max_seq_len, total_rows, sm_count, ctas_per_sm, chunk_len,
+                   num_splits);
+}
+
+gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes, int32_t* num_splits,
+                                     int32_t* chunk_len) {
+  Resolved r;
+  gqa_status st = resolve(params, &r, true);
+  if (st != GQA_OK) return st;
+  if (bytes) *bytes = r.bytes;
+  if (num_splits) *num_splits = r.S;
+  if (chunk_len) *chunk_len = r.chunk;
+  return GQA_OK;
+}
+
+gqa_status gqa_workspace_init(void* workspace, size_t workspace_bytes, gqa_stream_t stream) {
+  if (!workspace || workspace_bytes < kHeaderBytes) return GQA_ERR_WORKSPACE;
+  if (!is_device_ptr(workspace)) return GQA_ERR_DEVICE;
+  if (cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
   }
   return GQA_OK;
+}
+
+gqa_status gqa_decode_attend(const gqa_decode_params* p, gqa_stream_t stream) {
+  Resolved r;
+  gqa_status st = resolve(p, &r, true);
+  if (st != GQA_OK) return st;
+  if (!p->workspace || p->workspace_bytes < r.bytes) return GQA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
+  if (!is_device_ptr(p->workspace)) return GQA_ERR_DEVICE;
+  return attend_impl(p, r, static_cast<uint8_t*>(p->workspace), reinterpret_cast<cudaStream_t>(stream));
 }
 
 static gqa_status merge_common(const gqa_state* states, int32_t rows, int32_t num_states, int32_t head_dim,
@@ -465,10 +522,6 @@ static gqa_status merge_common(const gqa_state* states, int32_t rows, int32_t nu
   m.acc = num_states > 0 ? states->acc : nullptr;
   m.rows = rows;
   m.S = num_states;
-  m.offsets = nullptr;
-  m.H = 1;
-  m.chunk_len = 1;
-  m.max_len = 0;
   m.cm = has_carry ? carry_in->m : nullptr;
   m.cl = has_carry ? carry_in->l : nullptr;
   m.cacc = has_carry ? carry_in->acc : nullptr;
@@ -570,78 +623,14 @@ extern "C" gqa_status gqa_decode_attend_static_workspace(const gqa_decode_params
   }
   uint8_t* ws = static_cast<uint8_t*>(static_scratch_address(dev));
   if (ws == nullptr) return GQA_ERR_DEVICE;
-  const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out,
-                        p->carry_in.m, p->carry_in.l, p->carry_in.acc,
-                        p->state_out.m, p->state_out.l, p->state_out.acc,
-                        p->partials_out.m, p->partials_out.l, p->partials_out.acc};
-  for (const void* q : ptrs)
-    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
-  if (r.B == 0) return GQA_OK;
-
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  // The array keeps whatever the previous call left in it. Only the error word
-  // must start at zero (the partial states are written before they are read).
-  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), cs) != cudaSuccess) {
+  // The array keeps whatever the previous call left in it. The error word must
+  // start at zero; the segment tickets return to zero at the end of every
+  // completed call (and start at zero when the module loads); the partial
+  // states are written before they are read.
+  if (r.B > 0 && cudaMemsetAsync(ws, 0, sizeof(uint32_t), cs) != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_DEVICE;
   }
-  PartitionArgs a;
-  a.q = p->q;
-  a.k = p->k;
-  a.v = p->v;
-  a.offsets = p->offsets;
-  a.B = r.B;
-  a.H = r.H;
-  a.G = r.G;
-  a.hpk = r.hpk;
-  a.max_len = r.max_len;
-  a.chunk_len = r.chunk;
-  a.num_splits = r.S;
-  a.scale_log2 = r.scale * gqa::kLog2e;
-  if (r.has_partials) {
-    a.part_m = p->partials_out.m;
-    a.part_l = p->partials_out.l;
-    a.part_acc = p->partials_out.acc;
-    a.write_empty = 1;
-  } else {
-    a.part_m = reinterpret_cast<float*>(ws + r.off_m);
-    a.part_l = reinterpret_cast<float*>(ws + r.off_l);
-    a.part_acc = reinterpret_cast<float*>(ws + r.off_acc);
-    a.write_empty = 0;
-  }
-  a.err = reinterpret_cast<uint32_t*>(ws);
-
-  if (r.max_len > 0 || r.has_partials) {
-    CUtensorMap tk, tv;
-    const int map_rows = r.max_len > 0 ? r.max_len : 1;
-    const void* kb = r.max_len > 0 ? p->k : static_cast<const void*>(ws);
-    const void* vb = r.max_len > 0 ? p->v : static_cast<const void*>(ws);
-    if (r.bf16 && (!make_kv_map(&tk, kb, map_rows, r.G, r.D) || !make_kv_map(&tv, vb, map_rows, r.G, r.D)))
-      return GQA_ERR_DEVICE;
-    if (launch_partition(r, a, &tk, &tv, cs) != cudaSuccess) return GQA_ERR_DEVICE;
-  }
-  if (r.want_merge) {
-    MergeArgs m;
-    m.m = a.part_m;
-    m.l = a.part_l;
-    m.acc = a.part_acc;
-    m.rows = r.B * r.H;
-    m.S = r.S;
-    m.offsets = p->offsets;
-    m.H = r.H;
-    m.chunk_len = r.chunk;
-    m.max_len = r.max_len;
-    const bool has_carry = state_present(p->carry_in);
-    m.cm = has_carry ? p->carry_in.m : nullptr;
-    m.cl = has_carry ? p->carry_in.l : nullptr;
-    m.cacc = has_carry ? p->carry_in.acc : nullptr;
-    const bool has_so = state_present(p->state_out);
-    m.om = has_so ? p->state_out.m : nullptr;
-    m.ol = has_so ? p->state_out.l : nullptr;
-    m.oacc = has_so ? p->state_out.acc : nullptr;
-    m.out = p->out;
-    m.out_bf16 = r.out_bf16;
-    if (launch_merge_any(r.D, m, cs) != cudaSuccess) return GQA_ERR_DEVICE;
-  }
-  return GQA_OK;
+  return attend_impl(p, r, ws, cs);
 }

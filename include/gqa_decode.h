@@ -39,6 +39,8 @@
  *   - Dtypes: q/K/V are (fp32, fp32) or (bf16, bf16); any other pair is
  *     GQA_ERR_SHAPE_MISMATCH. Accumulation is fp32 in both cases.
  *   - head_dim is 64 or 128; heads per KV head (H / G) is 1..16.
+ *   - q, K, V, out and every acc array start on a 16-byte boundary
+ *     (GQA_ERR_SHAPE_MISMATCH otherwise).
  */
 #ifndef GQA_DECODE_H
 #define GQA_DECODE_H
@@ -134,14 +136,17 @@ typedef struct {
 gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes,
                                      int32_t* num_splits, int32_t* chunk_len);
 
-/* Zero the workspace's error word. Call once after allocating a workspace. */
+/* Zero a workspace (its error word and its per-sequence merge tickets). Call
+ * once after allocating a workspace, and again after a call reported
+ * GQA_ERR_TIMEOUT (an abandoned call can leave tickets behind). */
 gqa_status gqa_workspace_init(void* workspace, size_t workspace_bytes, gqa_stream_t stream);
 
 /* Decode attention with a mergeable online-softmax state ([attn.rs]
  * self_attn_incremental / cross_attn_incremental without the projections;
- * [usearch] § Attention with its carry). Launches the split-KV partition kernel
- * and, when out or state_out is requested, the merge/finalize kernel, on
- * `stream`. Asynchronous. */
+ * [usearch] § Attention with its carry). One kernel launch on `stream`: the
+ * split-KV partition kernel, whose last CTA per (sequence, KV head) merges that
+ * sequence's splits and the carry when out or state_out is requested.
+ * Asynchronous. */
 gqa_status gqa_decode_attend(const gqa_decode_params* params, gqa_stream_t stream);
 
 /* Decode attention exactly as gqa_decode_attend, for callers that cannot
@@ -196,11 +201,12 @@ gqa_status gqa_get_device_error(void* workspace, gqa_stream_t stream);
 
 /* The split plan of the heuristic, exposed for inspection and tests (host only):
  * chunk_len is a multiple of 64 and num_splits = ceil(max_seq_len / chunk_len).
- * total_rows is the expected sum of sequence lengths (<= batch*max_seq_len);
- * resident_ctas is the number of partition CTAs the GPU holds at once. */
+ * total_rows is the expected sum of sequence lengths (<= batch*max_seq_len;
+ * equal means every sequence has max_seq_len keys); sm_count and ctas_per_sm
+ * describe how many partition CTAs the GPU holds at once. */
 gqa_status gqa_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
-                           int64_t total_rows, int32_t resident_ctas, int32_t* chunk_len,
-                           int32_t* num_splits);
+                           int64_t total_rows, int32_t sm_count, int32_t ctas_per_sm,
+                           int32_t* chunk_len, int32_t* num_splits);
 
 /* Human-readable name of a status. Never NULL. */
 const char* gqa_status_string(gqa_status status);

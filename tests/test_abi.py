@@ -117,25 +117,36 @@ def test_workspace_init_refuses_small():
 
 def test_plan_uniform_configs():
     # 148 SMs x 2 resident CTAs
-    for B, G, N in [(16, 8, 4096), (4, 8, 32768), (1, 8, 131072), (1, 4, 512)]:
-        chunk, splits = gqa.gqa_plan_splits(B, G, N, B * N, 296)
+    for B, G, N in [(16, 8, 4096), (4, 8, 32768), (1, 8, 131072), (1, 4, 512), (64, 8, 4096),
+                    (3, 2, 1000)]:
+        chunk, splits = gqa.gqa_plan_splits(B, G, N, B * N, 148, 2)
         assert chunk % 64 == 0 and chunk >= 64
         assert splits == -(-N // chunk)
         assert (splits - 1) * chunk < N <= splits * chunk
-        if B * G * N >= 296 * 2 * 256:
-            # enough CTAs to fill every resident slot twice, each at least 256 rows
-            assert B * G * splits >= 296 and chunk >= 256
+        ctas = B * G * splits
+        # never a last wave that leaves most SMs idle
+        rem = ctas % 296
+        assert rem == 0 or rem >= 128 or ctas < 296
+
+
+def test_plan_matches_measured_best():
+    # split counts that measured fastest on B200 for these equal-length batches
+    assert gqa.gqa_plan_splits(16, 8, 4096, 16 * 4096, 148, 2) == (2048, 2)
+    assert 5 <= gqa.gqa_plan_splits(4, 8, 32768, 4 * 32768, 148, 2)[1] <= 9
+    assert gqa.gqa_plan_splits(1, 8, 131072, 131072, 148, 2)[1] in (18, 19, 37)
 
 
 def test_plan_ragged_uses_more_ctas():
-    c_u, s_u = gqa.gqa_plan_splits(64, 8, 16384, 64 * 16384, 296)
-    c_r, s_r = gqa.gqa_plan_splits(64, 8, 16384, 524320, 296)
+    c_u, s_u = gqa.gqa_plan_splits(64, 8, 16384, 64 * 16384, 148, 2)
+    c_r, s_r = gqa.gqa_plan_splits(64, 8, 16384, 524320, 148, 2)
     assert c_r <= c_u and s_r >= s_u
 
 
 def test_plan_degenerate():
-    assert gqa.gqa_plan_splits(0, 8, 100, 0, 296) == (64, 1)
-    assert gqa.gqa_plan_splits(3, 8, 0, 0, 296) == (64, 1)
-    assert gqa.gqa_plan_splits(1, 1, 1, 1, 296) == (64, 1)
+    assert gqa.gqa_plan_splits(0, 8, 100, 0) == (64, 1)
+    assert gqa.gqa_plan_splits(3, 8, 0, 0) == (64, 1)
+    assert gqa.gqa_plan_splits(1, 1, 1, 1) == (64, 1)
     with pytest.raises(gqa.GqaError):
-        gqa.gqa_plan_splits(1, 0, 10, 10, 296)
+        gqa.gqa_plan_splits(1, 0, 10, 10)
+    with pytest.raises(gqa.GqaError):
+        gqa.gqa_plan_splits(1, 1, 10, 10, 0, 2)
