@@ -861,31 +861,59 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
   const float* kg = static_cast<const float*>(a.k);
   const float* vg = static_cast<const float*>(a.v);
   const size_t rs = static_cast<size_t>(a.G) * D;
+  // U keys per warp step: their loads are issued together, their per-head dot
+  // products reduced together (U-way interleaved butterflies), and the running
+  // state rescaled once per step.
+  constexpr int U = 4;
 #pragma unroll 1
-  for (int key = t.kbeg + warp; key < t.kend; key += W) {
-    const size_t base = (static_cast<size_t>(t.o0) + key) * rs + static_cast<size_t>(t.g) * D + lane * E;
-    float kv[E], vv[E];
+  for (int key0 = t.kbeg + warp; key0 < t.kend; key0 += W * U) {
+    float kv[U][E], vv[U][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      kv[e] = __ldg(kg + base + e);
-      vv[e] = __ldg(vg + base + e);
+    for (int u = 0; u < U; ++u) {
+      const int key = key0 + u * W;
+      const bool live = key < t.kend;
+      const size_t base = (static_cast<size_t>(t.o0) + (live ? key : t.kbeg)) * rs +
+                          static_cast<size_t>(t.g) * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        kv[u][e] = live ? __ldg(kg + base + e) : 0.f;
+        vv[u][e] = live ? __ldg(vg + base + e) : 0.f;
+      }
     }
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
       if (h >= a.hpk) break;
-      float s = 0.f;
+      float sc[U];
 #pragma unroll
-      for (int e = 0; e < E; ++e) s = fmaf(qv[h][e], kv[e], s);
+      for (int u = 0; u < U; ++u) {
+        float d = 0.f;
 #pragma unroll
-      for (int x = 16; x >= 1; x >>= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
-      const float s2 = s * a.scale_log2;
-      const float mn = fmaxf(m[h], s2);
-      const float al = exp2f(m[h] - mn);
-      const float p = exp2f(s2 - mn);
-      l[h] = l[h] * al + p;
+        for (int e = 0; e < E; ++e) d = fmaf(qv[h][e], kv[u][e], d);
+        sc[u] = d;
+      }
 #pragma unroll
-      for (int e = 0; e < E; ++e) o[h][e] = fmaf(p, vv[e], o[h][e] * al);
-      m[h] = mn;
+      for (int x = 16; x >= 1; x >>= 1)
+#pragma unroll
+        for (int u = 0; u < U; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], x);
+      float mx = m[h];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        sc[u] = (key0 + u * W < t.kend) ? sc[u] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sc[u]);
+      }
+      const float al = exp2f(m[h] - mx);
+      float lsum = l[h] * al;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[h][e] *= al;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float p = exp2f(sc[u] - mx);
+        lsum += p;
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[h][e] = fmaf(p, vv[u][e], o[h][e]);
+      }
+      l[h] = lsum;
+      m[h] = mx;
     }
   }
   float* ms = fsm;

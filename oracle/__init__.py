@@ -52,7 +52,11 @@ def load(path=None):
     lib.oracle_decode_attend.argtypes = [
         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
         _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-        _f32p, _f32p, _f32p, _i64p, ctypes.c_int64, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+        _f32p, _f32p, _f32p, _f32p, _i64p, ctypes.c_int64, _f64p, _f64p, _f64p, _f64p,
+        ctypes.c_int]
+    lib.oracle_topk_to_bias.restype = ctypes.c_int
+    lib.oracle_topk_to_bias.argtypes = [_i32p, ctypes.c_int, ctypes.c_int, _i32p, _f32p,
+                                        ctypes.c_int64]
     lib.oracle_softmax_merge.restype = ctypes.c_int
     lib.oracle_softmax_merge.argtypes = [
         _f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
@@ -90,12 +94,14 @@ class State:
 
 
 def decode_attend(q, k, v, offsets, num_heads, num_kv_heads, score_scale=0.0,
-                  carry=None, rows=None, n_threads=0, lib=None):
+                  carry=None, rows=None, n_threads=0, lib=None, bias=None):
     """Exact decode attention in f64.
 
     q: [B, H, D]; k, v: [rows, G, D] (float32 or bf16 bits as uint16);
     offsets: int32 [B+1]; carry: optional (m [B*H], l [B*H], acc [B*H, D]) fp32;
-    rows: optional list of flat (b*H + h) rows to evaluate (default all).
+    rows: optional list of flat (b*H + h) rows to evaluate (default all);
+    bias: optional fp32 [rows of the cache], added to the scaled logit of each
+    cache row (-inf masks a key out).
     Returns a State whose arrays follow ``rows`` order.
     """
     lib = lib or load()
@@ -121,9 +127,11 @@ def decode_attend(q, k, v, offsets, num_heads, num_kv_heads, score_scale=0.0,
     cm = cl = cacc = None
     if carry is not None:
         cm, cl, cacc = (np.ascontiguousarray(c, dtype=np.float32) for c in carry)
+    bias_arr = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
     rc = lib.oracle_decode_attend(
         q.ctypes.data, q_bf16, k.ctypes.data, v.ctypes.data, kv_bf16, _ptr(offsets, _i32p),
-        B, H, G, D, float(score_scale), _ptr(cm, _f32p), _ptr(cl, _f32p), _ptr(cacc, _f32p),
+        B, H, G, D, float(score_scale), _ptr(bias_arr, _f32p),
+        _ptr(cm, _f32p), _ptr(cl, _f32p), _ptr(cacc, _f32p),
         _ptr(row_arr, _i64p), n, _ptr(om, _f64p), _ptr(ol, _f64p), _ptr(oacc, _f64p),
         _ptr(out, _f64p), int(n_threads))
     if rc != 0:
@@ -153,6 +161,41 @@ def softmax_merge(m, l, acc, carry=None, n_threads=0, lib=None):
     if rc != 0:
         raise ValueError("oracle_softmax_merge refused its arguments")
     return State(om, ol, oacc, out)
+
+
+def topk_to_bias(idx, offsets, rows, lib=None, fill=0.0):
+    """Additive bias per cache row from index rows idx [B, width] (int32,
+    positions relative to each sequence, -1 = INVALID): 0 for selected keys,
+    -inf for the other rows of each sequence, `fill` outside every sequence."""
+    lib = lib or load()
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    B = offsets.shape[0] - 1
+    width = idx.shape[1] if idx.ndim == 2 else 0
+    bias = np.full(int(rows), fill, np.float32)
+    rc = lib.oracle_topk_to_bias(_ptr(idx, _i32p), B, width, _ptr(offsets, _i32p),
+                                 _ptr(bias, _f32p), int(rows))
+    if rc != 0:
+        raise ValueError("oracle_topk_to_bias refused its arguments")
+    return bias
+
+
+def append_then_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_heads, score_scale=0.0,
+                       **kw):
+    """A decode step with the new token appended first (needle_core attn.rs:
+    KvCache::push_kv, then self_attn_incremental): row offsets[b+1]-1 of the
+    cache takes k_new[b], v_new[b]; then exact attention over the updated cache.
+    Returns (State, k_after, v_after) on host copies; the inputs are not modified."""
+    k2 = np.array(k, copy=True)
+    v2 = np.array(v, copy=True)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    for b in range(offsets.shape[0] - 1):
+        if offsets[b + 1] > offsets[b]:
+            k2[offsets[b + 1] - 1] = k_new[b]
+            v2[offsets[b + 1] - 1] = v_new[b]
+    st = decode_attend(q, k2, v2, offsets.astype(np.int32), num_heads, num_kv_heads, score_scale,
+                       **kw)
+    return st, k2, v2
 
 
 def bf16_to_f64(bits, lib=None):

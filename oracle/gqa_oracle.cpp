@@ -22,6 +22,11 @@
 //     out   = acc / l                                   (USearch § Attention:
 //             outputs already divided by the partition)
 //
+//   With an additive bias row (needle_core attn.rs `self_attn_incremental`,
+//   `attn_bias`: added to the scaled score of position t), the logit of key j
+//   is s_j = scale * q.k_j + bias[j], bias indexed by cache row; a bias of
+//   -inf masks the key out (weight 0).
+//
 //   The max-shifted exponentials follow the exact-softmax recipe of the
 //   cortiq_engine NystromState example `trial` (f64 exp of logit - max).
 //   A carry state with l == 0 is the empty state and contributes nothing,
@@ -73,6 +78,7 @@ struct AttendArgs {
   const int32_t* offsets;
   int B, H, G, D;
   double scale;
+  const float* bias;      // [rows] additive logit bias per cache row, or null
   const float* cm; const float* cl; const float* cacc;
   double* om; double* ol; double* oacc; double* out;
 };
@@ -114,6 +120,13 @@ void attend_one_row(const AttendArgs& a, int64_t row, int64_t r, std::vector<dou
 #else
     s[t] = a.scale * dot;
 #endif
+    if (a.bias != nullptr) {
+#if ORACLE_MUTATION == 9
+      s[t] = a.scale * (dot + static_cast<double>(a.bias[j]));   // bias inside the scale
+#else
+      s[t] += static_cast<double>(a.bias[j]);
+#endif
+    }
     if (s[t] > m) m = s[t];
   }
 
@@ -211,14 +224,14 @@ int oracle_default_threads(void) {
 // Returns 0 on success, -1 on a malformed argument.
 int oracle_decode_attend(const void* q, int q_bf16, const void* k, const void* v, int kv_bf16,
                          const int32_t* offsets, int B, int H, int G, int D, double score_scale,
-                         const float* cm, const float* cl, const float* cacc,
+                         const float* bias, const float* cm, const float* cl, const float* cacc,
                          const int64_t* row_list, int64_t n_rows, double* om, double* ol,
                          double* oacc, double* out, int n_threads) {
   if (B < 0 || H <= 0 || G <= 0 || D <= 0 || H % G != 0) return -1;
   if (!q || !k || !v || !offsets || !om || !ol || !oacc || !out) return -1;
   if ((cm == nullptr) != (cl == nullptr) || (cm == nullptr) != (cacc == nullptr)) return -1;
   AttendArgs a{q, q_bf16, k, v, kv_bf16, offsets, B, H, G, D,
-               score_scale != 0.0 ? score_scale : 1.0 / std::sqrt(static_cast<double>(D)),
+               score_scale != 0.0 ? score_scale : 1.0 / std::sqrt(static_cast<double>(D)), bias,
                cm, cl, cacc, om, ol, oacc, out};
   const int64_t total = static_cast<int64_t>(B) * H;
   const int64_t n = row_list ? n_rows : total;
@@ -279,6 +292,33 @@ int oracle_softmax_merge(const float* m, const float* l, const float* acc, int64
     ol[r] = L;
     for (int c = 0; c < D; ++c) out[r * D + c] = (L == 0.0) ? 0.0 : a[c] / L;
   });
+  return 0;
+}
+
+// Index-selected attention as a mask (metrale glm5next_dsa_ref, `topk_to_mask`:
+// the attention reads a visibility mask built from an index row; repeated
+// indices collapse, the INVALID sentinel -1 and out-of-range entries are
+// dropped). For decode, sequence b's index row idx[b, 0..width) holds key
+// positions relative to the sequence; the result is an additive bias per cache
+// row: 0 for a selected key of b, -inf for every other row of b. Rows outside
+// every sequence are left untouched.
+int oracle_topk_to_bias(const int32_t* idx, int B, int width, const int32_t* offsets, float* bias,
+                        int64_t rows) {
+  if (B < 0 || width < 0 || !offsets || !bias || (width > 0 && !idx)) return -1;
+  const float ninf = -std::numeric_limits<float>::infinity();
+  for (int b = 0; b < B; ++b) {
+    const int64_t o0 = offsets[b], o1 = offsets[b + 1];
+    if (o0 < 0 || o1 < o0 || o1 > rows) return -1;
+    for (int64_t r = o0; r < o1; ++r) bias[r] = ninf;
+    for (int w = 0; w < width; ++w) {
+      const int64_t t = idx[static_cast<int64_t>(b) * width + w];
+#if ORACLE_MUTATION == 10
+      if (t >= 0 && o0 + t <= o1) bias[o0 + t] = 0.0f;    // admits one past the end
+#else
+      if (t >= 0 && t < o1 - o0) bias[o0 + t] = 0.0f;
+#endif
+    }
+  }
   return 0;
 }
 

@@ -13,14 +13,19 @@ AssertionError when the oracle disagrees with:
     the KV heads permutes the outputs; merging the states of two disjoint key
     sets equals attending over their union; an empty carry changes nothing;
     adding a constant to every logit changes nothing; a planted high-logit key
-    dominates; ``score_scale = 0`` means ``1/sqrt(head_dim)``.
+    dominates; ``score_scale = 0`` means ``1/sqrt(head_dim)``;
+  * the additive bias row -- brute force with the bias added after the scale; a
+    constant bias only shifts m; a -inf bias equals removing the key; index rows
+    turned into a mask keep exactly the distinct in-range indices; appending a
+    token writes only its row and attends over it.
 
 Sources: needle_core ``attn.rs`` (``KvCache`` layout, ``self_attn_incremental``
 head map and scale); USearch linear algebra § Attention (online softmax folded
 into the walk, carry by partial-softmax rescaling, outputs divided by the
 partition, ``score_scale`` zero derives it); cortiq_engine ``NystromState``
 example ``trial`` (planted key); metrale glm5next_dsa_ref ``pool_states``
-(empty softmax gives 0, not NaN).
+(empty softmax gives 0, not NaN) and ``topk_to_mask`` (index rows -> mask);
+needle_core ``attn.rs`` ``attn_bias`` and ``KvCache::push_kv``.
 """
 import math
 
@@ -45,6 +50,10 @@ class OracleHandle:
     def bf16(self, bits):
         return self.pkg.bf16_to_f64(bits, lib=self.lib)
 
+    def topk_to_bias(self, *a, **kw):
+        kw.setdefault("lib", self.lib)
+        return self.pkg.topk_to_bias(*a, **kw)
+
 
 def _rng(seed):
     return np.random.default_rng(seed)
@@ -65,8 +74,9 @@ def _tiny(seed, lengths, H, G, D, scale=0.7):
     return q, k, v, _offsets(lengths)
 
 
-def brute_force(q, k, v, offsets, H, G, scale, carry=None):
-    """softmax(q K^T * scale) V per (b, h), matrix form, unshifted exp, in f64."""
+def brute_force(q, k, v, offsets, H, G, scale, carry=None, bias=None):
+    """softmax(q K^T * scale + bias) V per (b, h), matrix form, unshifted exp, in f64.
+    A bias of -inf gives its key weight exactly 0."""
     q = q.astype(np.float64)
     k = k.astype(np.float64)
     v = v.astype(np.float64)
@@ -80,6 +90,8 @@ def brute_force(q, k, v, offsets, H, G, scale, carry=None):
         k_h = np.repeat(kb, rep, axis=1)
         v_h = np.repeat(vb, rep, axis=1)
         logits = np.einsum("hd,nhd->hn", q[b], k_h) * scale        # [H, n]
+        if bias is not None:
+            logits = logits + np.asarray(bias, np.float64)[offsets[b]:offsets[b + 1]][None, :]
         w = np.exp(logits)
         num = np.einsum("hn,nhd->hd", w, v_h)
         den = w.sum(axis=1)
@@ -325,9 +337,78 @@ def pin_rows_subset(o):
     assert np.array_equal(sub.out, full.out[rows]) and np.array_equal(sub.m, full.m[rows])
 
 
+def pin_bias_brute_force(o):
+    # additive bias row after the scale (attn.rs attn_bias), incl. masked keys
+    for i, (lengths, H, G, D) in enumerate([([6, 9], 4, 2, 3), ([5, 0, 7], 6, 3, 4)]):
+        q, k, v, off = _tiny(1200 + i, lengths, H, G, D)
+        r = _rng(1300 + i)
+        bias = r.normal(0, 1, off[-1]).astype(np.float32)
+        bias[::4] = -np.inf
+        st = o.attend(q, k, v, off, H, G, score_scale=0.6, bias=bias)
+        _close(st.out, brute_force(q, k, v, off, H, G, 0.6, bias=bias), what=f"bias brute force {i}")
+
+
+def pin_bias_constant_is_shift(o):
+    q, k, v, off = _tiny(1400, [13, 4], 8, 2, 5)
+    base = o.attend(q, k, v, off, 8, 2, score_scale=0.4)
+    st = o.attend(q, k, v, off, 8, 2, score_scale=0.4, bias=np.full(off[-1], 7.5, np.float32))
+    _close(st.out, base.out, rtol=1e-13, atol=1e-14, what="constant bias")
+    _close(st.m, base.m + 7.5, rtol=1e-14, what="constant bias shifts m")
+
+
+def pin_bias_mask_is_subset(o):
+    # masking rows with -inf equals attending over the cache without them
+    H, G, D = 4, 2, 4
+    q, k, v, off = _tiny(1500, [10, 6], H, G, D)
+    keep = np.ones(off[-1], bool)
+    keep[[1, 2, 7, 11, 15]] = False
+    bias = np.where(keep, 0.0, -np.inf).astype(np.float32)
+    st = o.attend(q, k, v, off, H, G, bias=bias)
+    sub_off = np.array([0, keep[:10].sum(), keep.sum()], np.int32)
+    ref = o.attend(q, k[keep], v[keep], sub_off, H, G)
+    assert np.array_equal(st.out, ref.out) and np.array_equal(st.l, ref.l), "mask = subset"
+    # every key of a sequence masked: weight 0, output 0 (or the carry alone)
+    bias[:10] = -np.inf
+    st = o.attend(q, k, v, off, H, G, bias=bias)
+    assert np.all(st.out[:H] == 0.0) and np.all(np.isneginf(st.m[:H]))
+
+
+def pin_topk_to_bias(o):
+    # index rows: repeated indices collapse, -1 (INVALID) and out-of-range entries drop
+    off = np.array([0, 5, 5, 12], np.int32)
+    idx = np.array([[4, 0, 4, -1, 5, 2],
+                    [0, 1, -1, -1, -1, -1],
+                    [6, 6, 7, -3, 3, 0]], np.int32)
+    bias = o.topk_to_bias(idx, off, 14, fill=1.25)
+    for b in range(3):
+        n = off[b + 1] - off[b]
+        selected = {int(t) for t in idx[b] if 0 <= t < n}
+        for t in range(n):
+            want = 0.0 if t in selected else -np.inf
+            assert bias[off[b] + t] == want, f"topk bias seq {b} key {t}"
+    assert np.all(bias[12:] == 1.25), "rows outside every sequence are left alone"
+
+
+def pin_append_then_attend(o):
+    H, G, D = 4, 2, 3
+    q, k, v, off = _tiny(1600, [5, 1, 3], H, G, D)
+    r = _rng(1601)
+    kn = r.uniform(-1, 1, (3, G, D)).astype(np.float32)
+    vn = r.uniform(-1, 1, (3, G, D)).astype(np.float32)
+    st, k2, v2 = o.pkg.append_then_attend(q, k, v, off, kn, vn, H, G, lib=o.lib)
+    for b in range(3):
+        assert np.array_equal(k2[off[b + 1] - 1], kn[b]) and np.array_equal(v2[off[b + 1] - 1], vn[b])
+    untouched = np.ones(off[-1], bool)
+    untouched[off[1:] - 1] = False
+    assert np.array_equal(k2[untouched], k[untouched]), "append touched other rows"
+    _close(st.out, brute_force(q, k2, v2, off, H, G, 1 / math.sqrt(D)), what="append then attend")
+
+
 ALL_PINS = [pin_bf16_widening, pin_brute_force_tiny, pin_single_key, pin_constant_v,
             pin_zero_query_mean, pin_two_key_closed_form, pin_group_symmetry, pin_merge_union,
-            pin_carry_identity, pin_shift_invariance, pin_needle, pin_rows_subset]
+            pin_carry_identity, pin_shift_invariance, pin_needle, pin_rows_subset,
+            pin_bias_brute_force, pin_bias_constant_is_shift, pin_bias_mask_is_subset,
+            pin_topk_to_bias, pin_append_then_attend]
 
 
 def run_all(o):

@@ -3,7 +3,8 @@
 Every ORACLE_MUTATION build in oracle/gqa_oracle.cpp is a plausible slip: an
 interleaved head map, a dropped scale, a carry rescaled with the wrong sign, an
 output not divided by the partition, a transposed cache layout, partial states
-merged without rescaling, a dropped last key, keys used as values.
+merged without rescaling, a dropped last key, keys used as values, a bias added
+before the scale, a top-k index one past a sequence's end accepted.
 """
 import os
 
@@ -15,7 +16,8 @@ from oracle import build as oracle_build
 
 MUTATIONS = {1: "interleaved head map", 2: "scale dropped", 3: "carry sign flipped",
              4: "not divided by partition", 5: "cache layout transposed",
-             6: "merge without rescaling", 7: "last key dropped", 8: "keys used as values"}
+             6: "merge without rescaling", 7: "last key dropped", 8: "keys used as values",
+             9: "bias inside the scale", 10: "top-k admits one past the end"}
 
 
 @pytest.mark.parametrize("mutation", sorted(MUTATIONS), ids=lambda m: MUTATIONS[m])
