@@ -6,9 +6,10 @@ provides device memory (the tensors passed in, and outputs/workspace allocated
 here when the caller gives none) and the current CUDA stream.
 
 The entry points keep the C names:
-  gqa_decode_attend, gqa_decode_workspace_size, gqa_workspace_init,
-  gqa_softmax_merge, gqa_state_finalize, gqa_get_device_error,
-  gqa_plan_splits, gqa_status_string, gqa_version.
+  gqa_decode_attend, gqa_decode_append_attend, gqa_topk_to_bias,
+  gqa_decode_workspace_size, gqa_workspace_init, gqa_softmax_merge,
+  gqa_state_finalize, gqa_get_device_error, gqa_plan_splits,
+  gqa_status_string, gqa_version, gqa_decode_attend_static_workspace.
 
 If the compiled library is missing the first call raises ``LibraryMissing``;
 there is no fallback implementation.
@@ -19,6 +20,7 @@ import os
 
 __all__ = [
     "GqaError", "LibraryMissing", "State", "Workspace", "gqa_decode_attend",
+    "gqa_decode_append_attend", "gqa_topk_to_bias", "gqa_decode_attend_static_workspace",
     "gqa_decode_workspace_size", "gqa_workspace_init", "gqa_softmax_merge", "gqa_state_finalize",
     "gqa_get_device_error", "gqa_plan_splits", "gqa_status_string", "gqa_version", "lib_path",
     "load_library",
@@ -66,6 +68,7 @@ class _CParams(ctypes.Structure):
         ("partials_out", _CState),
         ("num_splits", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("bias", ctypes.c_void_p),
     ]
 
 
@@ -93,6 +96,8 @@ def load_library(path=None):
                                               ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.gqa_workspace_init.argtypes = [sp, ctypes.c_size_t, sp]
     lib.gqa_decode_attend.argtypes = [ctypes.POINTER(_CParams), sp]
+    lib.gqa_decode_append_attend.argtypes = [ctypes.POINTER(_CParams), sp, sp, sp]
+    lib.gqa_topk_to_bias.argtypes = [sp, i32, i32, sp, i32, sp, sp, sp]
     lib.gqa_softmax_merge.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
     lib.gqa_state_finalize.argtypes = [ps, i32, i32, sp, i32, sp]
     lib.gqa_get_device_error.argtypes = [sp, sp]
@@ -101,7 +106,8 @@ def load_library(path=None):
     lib.gqa_status_string.restype = ctypes.c_char_p
     lib.gqa_version.argtypes = []
     for fn in ("gqa_decode_workspace_size", "gqa_workspace_init", "gqa_decode_attend", "gqa_softmax_merge",
-               "gqa_state_finalize", "gqa_get_device_error", "gqa_plan_splits"):
+               "gqa_state_finalize", "gqa_get_device_error", "gqa_plan_splits",
+               "gqa_decode_append_attend", "gqa_topk_to_bias"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gqa_version.restype = ctypes.c_int32
     if path is None:
@@ -220,7 +226,7 @@ def _default_workspace(device):
 
 
 def _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out,
-            out_dtype, partials_out, num_splits, max_seq_len, max_len):
+            out_dtype, partials_out, num_splits, max_seq_len, max_len, bias=None):
     p = _CParams()
     p.struct_size = ctypes.sizeof(_CParams)
     p.q, p.q_dtype = _ptr(q), _dtype_code(q)
@@ -241,6 +247,11 @@ def _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state
     p.out_dtype = out_dtype
     p.partials_out = _c_state(partials_out)
     p.num_splits = int(num_splits)
+    if bias is not None:
+        torch = _torch()
+        if bias.dtype != torch.float32:
+            raise GqaError(GQA_ERR_SHAPE_MISMATCH, "bias must be float32")
+    p.bias = _ptr(bias)
     return p
 
 
@@ -262,16 +273,9 @@ def gqa_decode_workspace_size(q, k, v, offsets, num_heads, num_kv_heads=0, *, sc
     return nbytes.value, ns.value, cl.value
 
 
-def gqa_decode_attend(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scale=0.0, carry=None,
-                      state_out=None, out=None, out_dtype=None, partials_out=None, want_out=None,
-                      num_splits=0, max_seq_len=0, max_len=None, workspace=None, stream=None):
-    """Decode attention over a KV cache; see include/gqa_decode.h.
-
-    q [B, H, D]; k, v [max_len, G, D]; offsets int32 [B+1] on the device.
-    carry / state_out / partials_out: ``State`` objects or None. ``out`` is
-    allocated ([B, H, D], out_dtype or q's dtype) unless given, or unless only
-    state_out / partials_out are wanted (want_out=False). Returns out (or None).
-    """
+def _attend_call(entry, q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out,
+                 out_dtype, partials_out, want_out, num_splits, max_seq_len, max_len, workspace, stream,
+                 bias, extra=()):
     torch = _torch()
     if want_out is None:
         want_out = out is not None or (state_out is None and partials_out is None)
@@ -282,7 +286,7 @@ def gqa_decode_attend(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scal
     if out is not None:
         odt = _dtype_code(out)
     p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
-                partials_out, num_splits, max_seq_len, max_len)
+                partials_out, num_splits, max_seq_len, max_len, bias)
     lib = load_library()
     nbytes = ctypes.c_size_t()
     _check(lib.gqa_decode_workspace_size(ctypes.byref(p), ctypes.byref(nbytes), None, None),
@@ -291,8 +295,56 @@ def gqa_decode_attend(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scal
     ws.reserve(nbytes.value, stream)
     p.workspace = ws.ptr
     p.workspace_bytes = ws.nbytes
-    _check(lib.gqa_decode_attend(ctypes.byref(p), _stream_handle(stream)), "gqa_decode_attend")
+    _check(getattr(lib, entry)(ctypes.byref(p), *extra, _stream_handle(stream)), entry)
     return out
+
+
+def gqa_decode_attend(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scale=0.0, carry=None,
+                      state_out=None, out=None, out_dtype=None, partials_out=None, want_out=None,
+                      num_splits=0, max_seq_len=0, max_len=None, workspace=None, stream=None,
+                      bias=None):
+    """Decode attention over a KV cache; see include/gqa_decode.h.
+
+    q [B, H, D]; k, v [max_len, G, D]; offsets int32 [B+1] on the device.
+    carry / state_out / partials_out: ``State`` objects or None. ``out`` is
+    allocated ([B, H, D], out_dtype or q's dtype) unless given, or unless only
+    state_out / partials_out are wanted (want_out=False). bias: optional fp32
+    [max_len] additive logit bias per cache row. Returns out (or None).
+    """
+    return _attend_call("gqa_decode_attend", q, k, v, offsets, num_heads, num_kv_heads, score_scale,
+                        carry, state_out, out, out_dtype, partials_out, want_out, num_splits,
+                        max_seq_len, max_len, workspace, stream, bias)
+
+
+def gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_heads=0, *,
+                             score_scale=0.0, carry=None, state_out=None, out=None, out_dtype=None,
+                             want_out=None, num_splits=0, max_seq_len=0, max_len=None,
+                             workspace=None, stream=None, bias=None):
+    """Append k_new/v_new [B, G, D] at row offsets[b+1]-1 of the caches (which
+    are written), then attend with the new key included; see include/gqa_decode.h."""
+    if k_new.dtype != k.dtype or v_new.dtype != k.dtype:
+        raise GqaError(GQA_ERR_SHAPE_MISMATCH, "k_new/v_new must have the cache dtype")
+    return _attend_call("gqa_decode_append_attend", q, k, v, offsets, num_heads, num_kv_heads,
+                        score_scale, carry, state_out, out, out_dtype, None, want_out, num_splits,
+                        max_seq_len, max_len, workspace, stream, bias,
+                        extra=(ctypes.c_void_p(_ptr(k_new)), ctypes.c_void_p(_ptr(v_new))))
+
+
+def gqa_topk_to_bias(idx, offsets, max_len, bias=None, workspace=None, stream=None):
+    """fp32 bias [max_len] from index rows idx [B, width] (int32, relative key
+    positions, -1 = INVALID): selected keys 0, the sequences' other rows -inf.
+    Rows outside every sequence keep their value (0 when bias is allocated here)."""
+    torch = _torch()
+    if bias is None:
+        bias = torch.zeros(int(max_len), dtype=torch.float32, device=offsets.device)
+    B = offsets.numel() - 1
+    width = idx.shape[1] if idx.dim() == 2 else 0
+    _check(load_library().gqa_topk_to_bias(ctypes.c_void_p(_ptr(idx)), B, width,
+                                           ctypes.c_void_p(_ptr(offsets)), int(max_len),
+                                           ctypes.c_void_p(_ptr(bias)),
+                                           ctypes.c_void_p(workspace.ptr) if workspace else None,
+                                           _stream_handle(stream)), "gqa_topk_to_bias")
+    return bias
 
 
 def gqa_softmax_merge(states, carry=None, merged_out=None, out=None, out_dtype=None, want_out=None,

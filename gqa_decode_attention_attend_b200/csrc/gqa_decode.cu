@@ -268,6 +268,7 @@ gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
       reinterpret_cast<uintptr_t>(p->carry_in.acc) | reinterpret_cast<uintptr_t>(p->state_out.acc) |
       reinterpret_cast<uintptr_t>(p->partials_out.acc);
   if (align_or & 15u) return GQA_ERR_SHAPE_MISMATCH;
+  if (reinterpret_cast<uintptr_t>(p->bias) & 3u) return GQA_ERR_SHAPE_MISMATCH;
   if (!std::isfinite(p->score_scale)) return GQA_ERR_INVALID_ARGUMENT;
   r->scale = p->score_scale != 0.f ? p->score_scale : 1.0f / sqrtf(static_cast<float>(r->D));
   if (static_cast<int64_t>(r->B) * r->H * r->D > INT32_MAX) return GQA_ERR_INVALID_ARGUMENT;
@@ -370,11 +371,13 @@ cudaError_t launch_partition(const Resolved& r, const PartitionArgs& a, const CU
 
 // Pointer checks and the single launch of a decode call, with the scratch at `ws`
 // (the caller's workspace, or the library's static array).
-gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* ws, cudaStream_t cs) {
+gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* ws, cudaStream_t cs,
+                       const void* k_new = nullptr, const void* v_new = nullptr) {
   const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out,
                         p->carry_in.m, p->carry_in.l, p->carry_in.acc,
                         p->state_out.m, p->state_out.l, p->state_out.acc,
-                        p->partials_out.m, p->partials_out.l, p->partials_out.acc};
+                        p->partials_out.m, p->partials_out.l, p->partials_out.acc,
+                        p->bias, k_new, v_new};
   for (const void* q : ptrs)
     if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
   if (r.B == 0) return GQA_OK;
@@ -416,6 +419,12 @@ gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* w
   a.oacc = has_so ? p->state_out.acc : nullptr;
   a.out = p->out;
   a.out_bf16 = r.out_bf16;
+  a.bias = p->bias;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.kw = const_cast<void*>(p->k);
+  a.vw = const_cast<void*>(p->v);
+  a.kv_elem = r.bf16 ? 2 : 4;
 
   // With no cache rows every tile is empty and no load is issued, but a tensor
   // map still needs a non-zero extent and a valid aligned base: the scratch
@@ -489,6 +498,36 @@ gqa_status gqa_decode_attend(const gqa_decode_params* p, gqa_stream_t stream) {
   if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
   if (!is_device_ptr(p->workspace)) return GQA_ERR_DEVICE;
   return attend_impl(p, r, static_cast<uint8_t*>(p->workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+gqa_status gqa_decode_append_attend(const gqa_decode_params* p, const void* k_new, const void* v_new,
+                                    gqa_stream_t stream) {
+  Resolved r;
+  gqa_status st = resolve(p, &r, true);
+  if (st != GQA_OK) return st;
+  if (r.B > 0 && (!k_new || !v_new || r.max_len == 0)) return GQA_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u)
+    return GQA_ERR_SHAPE_MISMATCH;
+  if (!p->workspace || p->workspace_bytes < r.bytes) return GQA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
+  if (!is_device_ptr(p->workspace)) return GQA_ERR_DEVICE;
+  return attend_impl(p, r, static_cast<uint8_t*>(p->workspace), reinterpret_cast<cudaStream_t>(stream),
+                     k_new, v_new);
+}
+
+gqa_status gqa_topk_to_bias(const int32_t* idx, int32_t batch, int32_t width, const int32_t* offsets,
+                            int32_t max_len, float* bias, void* workspace, gqa_stream_t stream) {
+  if (batch < 0 || width < 0 || max_len < 0) return GQA_ERR_INVALID_ARGUMENT;
+  if (batch == 0) return GQA_OK;
+  if (!offsets || !bias || (width > 0 && !idx)) return GQA_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(bias) & 3u) return GQA_ERR_SHAPE_MISMATCH;
+  const void* ptrs[] = {idx, offsets, bias, workspace};
+  for (const void* q : ptrs)
+    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
+  gqa::gqa_topk_to_bias_kernel<<<batch, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      idx, width, offsets, max_len, bias, static_cast<uint32_t*>(workspace));
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_DEVICE;
+  return GQA_OK;
 }
 
 static gqa_status merge_common(const gqa_state* states, int32_t rows, int32_t num_states, int32_t head_dim,

@@ -66,6 +66,18 @@ struct PartitionArgs {
   float* oacc;
   void* out;                 // [B*H, D] or null
   int32_t out_bf16;
+  // Additive logit bias per cache row (fp32 [max_len], natural-log units, -inf
+  // masks the key), or null (needle_core attn.rs, self_attn_incremental: attn_bias).
+  const float* bias;
+  // Append (needle_core attn.rs, KvCache::push_kv before the attention): when
+  // k_new is set, the new token of sequence b is its last key, row
+  // offsets[b+1]-1: the CTA owning that key writes k_new/v_new [B, G, D] into
+  // kw/vw (the caches) and folds the key in from k_new/v_new directly.
+  const void* k_new;
+  const void* v_new;
+  void* kw;
+  void* vw;
+  int32_t kv_elem;           // bytes per cache element (2 or 4)
 };
 
 // Work item of a CTA: flattened index -> (b, split c, g), g fastest so that the
@@ -75,6 +87,8 @@ struct Tile {
   int o0;           // first cache row of the sequence
   int n;            // keys of the sequence (0 if its offsets are malformed)
   int kbeg, kend;   // key range of the tile, relative to the sequence
+  int kstream;      // end of the keys read from the cache (kend, or n-1 for the append tile)
+  bool append;      // this tile owns the appended (last) key of the sequence
 };
 
 __device__ __forceinline__ Tile tile_of(const PartitionArgs& a, int bid) {
@@ -94,7 +108,43 @@ __device__ __forceinline__ Tile tile_of(const PartitionArgs& a, int bid) {
   t.n = n;
   t.kbeg = t.c * a.chunk_len;
   t.kend = (t.c == a.num_splits - 1) ? n : min(n, t.kbeg + a.chunk_len);
+  t.append = a.k_new != nullptr && t.kbeg < t.kend && t.kend == n;
+  t.kstream = t.append ? n - 1 : t.kend;
+  if (a.k_new != nullptr && n == 0 && t.c == 0 && t.g == 0 && threadIdx.x == 0)
+    atomicOr(a.err, kErrBadOffsets);     // no row for the appended token
   return t;
+}
+
+// Logit bias of key `key` (relative to the sequence) in base-2 units.
+__device__ __forceinline__ float bias2(const PartitionArgs& a, const Tile& t, int key) {
+  return a.bias != nullptr ? __ldg(a.bias + t.o0 + key) * kLog2e : 0.f;
+}
+
+// Append tile: copy the new token's K and V rows of head g into the caches.
+__device__ __forceinline__ void write_appended_row(const PartitionArgs& a, const Tile& t, int D,
+                                                   int tid, int nthreads) {
+  const size_t row_bytes = static_cast<size_t>(D) * a.kv_elem;
+  const size_t src = (static_cast<size_t>(t.b) * a.G + t.g) * row_bytes;
+  const size_t dst = ((static_cast<size_t>(t.o0) + t.n - 1) * a.G + t.g) * row_bytes;
+  const int chunks = static_cast<int>(row_bytes / 16);
+  for (int i = tid; i < 2 * chunks; i += nthreads) {
+    const bool isv = i >= chunks;
+    const int j = isv ? i - chunks : i;
+    const uint4 val = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(isv ? a.v_new : a.k_new) + src + 16 * j);
+    *reinterpret_cast<uint4*>(static_cast<uint8_t*>(isv ? a.vw : a.kw) + dst + 16 * j) = val;
+  }
+}
+
+// Base-2 logit of the appended key for query head h of the tile's group,
+// computed by one warp (lanes split D); q and k_new in the cache dtype.
+template <int D, typename T>
+__device__ __forceinline__ float appended_logit2(const PartitionArgs& a, const Tile& t, int h, int lane) {
+  const T* q = static_cast<const T*>(a.q) + (static_cast<size_t>(t.b) * a.H + static_cast<size_t>(t.g) * a.hpk + h) * D;
+  const T* k = static_cast<const T*>(a.k_new) + (static_cast<size_t>(t.b) * a.G + t.g) * D;
+  float s = 0.f;
+  for (int d = lane; d < D; d += 32) s = fmaf(static_cast<float>(q[d]), static_cast<float>(k[d]), s);
+  for (int x = 16; x >= 1; x >>= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
+  return s * a.scale_log2 + bias2(a, t, t.n - 1);
 }
 
 __device__ __forceinline__ size_t state_index(const PartitionArgs& a, const Tile& t, int h) {
@@ -115,28 +165,32 @@ __device__ __forceinline__ void write_empty_states(const PartitionArgs& a, const
 }
 
 // Cross-warp combine of per-warp states held in shared memory, then store of the
-// tile's partial state. ms/ls: [W][HP] base-2 maxima and partitions; accs:
-// [W][HP][D + 4], already rescaled to the tile maximum. Threads 0..nthreads-1.
+// tile's partial state. ms/ls: [nslots][HP] base-2 maxima and partitions; accs:
+// [nslots][HP][D + 4], already rescaled to the tile maximum; nslots is W, or
+// W + 1 when the appended key occupies an extra slot. Threads 0..nthreads-1.
 template <int D, int W, int HP>
 __device__ __forceinline__ void store_partial(const PartitionArgs& a, const Tile& t,
                                               const float* ms, const float* ls, const float* accs,
-                                              int tid, int nthreads) {
+                                              int tid, int nthreads, int nslots = W) {
   constexpr int P = D + 4;
   for (int i = tid; i < a.hpk * D; i += nthreads) {
     const int h = i / D, d = i % D;
     float s = 0.f;
 #pragma unroll
-    for (int w = 0; w < W; ++w) s += accs[(w * HP + h) * P + d];
+    for (int w = 0; w < W + 1; ++w)
+      if (w < nslots) s += accs[(w * HP + h) * P + d];
     a.part_acc[state_index(a, t, h) * D + d] = s;
   }
   for (int h = tid; h < a.hpk; h += nthreads) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < W; ++w) M = fmaxf(M, ms[w * HP + h]);
+    for (int w = 0; w < W + 1; ++w)
+      if (w < nslots) M = fmaxf(M, ms[w * HP + h]);
     const float Mu = (M == -INFINITY) ? 0.f : M;
     float L = 0.f;
 #pragma unroll
-    for (int w = 0; w < W; ++w) L += ls[w * HP + h] * exp2f(ms[w * HP + h] - Mu);
+    for (int w = 0; w < W + 1; ++w)
+      if (w < nslots) L += ls[w * HP + h] * exp2f(ms[w * HP + h] - Mu);
     const size_t s = state_index(a, t, h);
     a.part_m[s] = (L == 0.f) ? -INFINITY : M * kLn2;
     a.part_l[s] = L;
@@ -503,13 +557,13 @@ struct TcCfg {
   static constexpr int kStages = (D == 128) ? 3 : 4;
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kHP = 8 * NT;                                // padded heads
-  static constexpr int kScratchBytes = kConsumerWarps * kHP * (D + 4 + 2) * 4;
+  static constexpr int kScratchBytes = (kConsumerWarps + 1) * kHP * (D + 4 + 2) * 4;
   static constexpr int kDataBytes = kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes;
   static constexpr int kBarOffset = kDataBytes;                     // 2*kStages + 1 mbarriers
   static constexpr int kAbortOffset = kBarOffset + (2 * kStages + 1 + 1) * 8;
   static constexpr int kFlagOffset = kAbortOffset + 4;
-  static constexpr int kMergeOffset = kAbortOffset + 16;            // 3 x 16 floats
-  static constexpr int kSmemBytes = 1024 + kMergeOffset + 3 * 16 * 4;   // + alignment slack
+  static constexpr int kMergeOffset = kAbortOffset + 16;            // 4 x 16 floats
+  static constexpr int kSmemBytes = 1024 + kMergeOffset + 4 * 16 * 4;   // + alignment slack
   // The merge's split weights reuse the ring (idle once the tile is consumed).
   static constexpr int kWeightCap = kRingBytes / 4 / 2;
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
@@ -537,6 +591,7 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   float* smM = reinterpret_cast<float*>(smem + C::kMergeOffset);
   float* smL = smM + 16;
   float* smC = smM + 32;
+  float* smN = smM + 48;                         // appended key's base-2 logit per head
   int* smFlag = reinterpret_cast<int*>(smem + C::kFlagOffset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -549,7 +604,7 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
                                C::kWeightCap, NamedSync128{});
     return;
   }
-  const int nst = (t.kend - t.kbeg + C::kStageKeys - 1) / C::kStageKeys;
+  const int nst = (t.kstream - t.kbeg + C::kStageKeys - 1) / C::kStageKeys;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -638,6 +693,13 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
   const float sl2 = a.scale_log2;
   bool aborted = false;
+  if (t.append) {
+    write_appended_row(a, t, D, threadIdx.x, 32 * C::kConsumerWarps);
+    for (int h = warp; h < a.hpk; h += C::kConsumerWarps) {
+      const float s2 = appended_logit2<D, __nv_bfloat16>(a, t, h, lane);
+      if (lane == 0) smN[h] = s2;
+    }
+  }
 
 #pragma unroll 1
   for (int it = 0; it < nst; ++it) {
@@ -650,7 +712,7 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     if (aborted) break;
     const int key0 = t.kbeg + it * C::kStageKeys + warp * C::kKeysPerWarp;
-    const int nvalid = min(C::kKeysPerWarp, t.kend - key0);
+    const int nvalid = min(C::kKeysPerWarp, t.kstream - key0);
     const uint32_t kt = ring + s * C::kStageBytes;
     const uint32_t vt = kt + C::kHalves * C::kHalfTileBytes;
     const int wrow = warp * C::kKeysPerWarp;
@@ -689,6 +751,8 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
       // Online softmax update (base 2). Fragment: sacc[nt][e] is key lane/4,
       // sacc[nt][e+2] key lane/4+8, both for head column nt*8 + 2*(lane%4) + e.
       const int kr = lane >> 2;
+      const float b0 = (kr < nvalid) ? bias2(a, t, key0 + kr) : 0.f;
+      const float b1 = (kr + 8 < nvalid) ? bias2(a, t, key0 + kr + 8) : 0.f;
       uint32_t ph_hi[NT][2], ph_lo[NT][2];
       float alpha[NT][2];
 #pragma unroll
@@ -696,8 +760,8 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
         float p[4];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float s0 = (kr < nvalid) ? sacc[nt][e] * sl2 : -INFINITY;
-          const float s1 = (kr + 8 < nvalid) ? sacc[nt][e + 2] * sl2 : -INFINITY;
+          const float s0 = (kr < nvalid) ? fmaf(sacc[nt][e], sl2, b0) : -INFINITY;
+          const float s1 = (kr + 8 < nvalid) ? fmaf(sacc[nt][e + 2], sl2, b1) : -INFINITY;
           float mx = fmaxf(s0, s1);
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -767,9 +831,11 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   constexpr int W = C::kConsumerWarps, HP = C::kHP, P = D + 4;
   const int ctid = threadIdx.x;                   // 0 .. 32*W-1
   ptx::named_barrier_sync(1, 32 * W);             // ring no longer read by anyone
+  // slots: W warps, plus the appended key when this tile owns it
   float* ms = reinterpret_cast<float*>(smem);
-  float* ls = ms + W * HP;
-  float* accs = ls + W * HP;
+  float* ls = ms + (W + 1) * HP;
+  float* accs = ls + (W + 1) * HP;
+  const int nslots = W + (t.append ? 1 : 0);
   if (lane < 4) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -779,6 +845,11 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
         ls[warp * HP + nt * 8 + lane * 2 + e] = lrun[nt][e];
       }
   }
+  if (t.append)   // the appended key as one more slot: m = its logit, l = 1
+    for (int h = ctid; h < HP; h += 32 * W) {
+      ms[W * HP + h] = h < a.hpk ? smN[h] : -INFINITY;
+      ls[W * HP + h] = h < a.hpk ? 1.f : 0.f;
+    }
   ptx::named_barrier_sync(1, 32 * W);
   float f[NT][2];
 #pragma unroll
@@ -788,9 +859,19 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
       const int hc = nt * 8 + (lane & 3) * 2 + e;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < W; ++w) M = fmaxf(M, ms[w * HP + hc]);
+      for (int w = 0; w < W + 1; ++w)
+        if (w < nslots) M = fmaxf(M, ms[w * HP + hc]);
       const float Mu = (M == -INFINITY) ? 0.f : M;
       f[nt][e] = exp2f(mrun[nt][e] - Mu);
+    }
+  if (t.append)
+    for (int i = ctid; i < a.hpk * D; i += 32 * W) {
+      const int h = i / D, d = i % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < W + 1; ++w) M = fmaxf(M, ms[w * HP + h]);
+      const float vn = __bfloat162float(static_cast<const __nv_bfloat16*>(a.v_new)[(static_cast<size_t>(t.b) * a.G + t.g) * D + d]);
+      accs[(W * HP + h) * P + d] = vn * exp2f(ms[W * HP + h] - (M == -INFINITY ? 0.f : M));
     }
 #pragma unroll
   for (int mt = 0; mt < D / 16; ++mt)
@@ -805,7 +886,7 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
   ptx::named_barrier_sync(1, 32 * W);
   if (*abort_flag) return;
-  store_partial<D, W, HP>(a, t, ms, ls, accs, ctid, 32 * W);
+  store_partial<D, W, HP>(a, t, ms, ls, accs, ctid, 32 * W, nslots);
   static_assert(C::kConsumerWarps == 4, "NamedSync128 spans the four consumer warps");
   if (a.merge) {
     ptx::named_barrier_sync(1, 32 * W);     // store_partial done with the ring scratch
@@ -823,7 +904,7 @@ struct F32Cfg {
   static constexpr int kWarps = 4;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kE = D / 32;  // elements per lane
-  static constexpr int kSmemBytes = kWarps * HMAX * (D + 4 + 2) * 4;
+  static constexpr int kSmemBytes = (kWarps + 1) * HMAX * (D + 4 + 2) * 4;
   static constexpr int kWeightCap = kSmemBytes / 4 / 2;
 };
 
@@ -833,7 +914,7 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
   using C = F32Cfg<D, HMAX>;
   constexpr int E = C::kE, W = C::kWarps, HP = HMAX, P = D + 4;
   extern __shared__ float fsm[];
-  __shared__ float smM[16], smL[16], smC[16];
+  __shared__ float smM[16], smL[16], smC[16], smN[16];
   __shared__ int smFlag;
   const Tile t = tile_of(a, blockIdx.x);
   if (t.kbeg >= t.kend) {
@@ -861,17 +942,24 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
   const float* kg = static_cast<const float*>(a.k);
   const float* vg = static_cast<const float*>(a.v);
   const size_t rs = static_cast<size_t>(a.G) * D;
+  if (t.append) {
+    write_appended_row(a, t, D, threadIdx.x, C::kThreads);
+    for (int h = warp; h < a.hpk; h += W) {
+      const float s2 = appended_logit2<D, float>(a, t, h, lane);
+      if (lane == 0) smN[h] = s2;
+    }
+  }
   // U keys per warp step: their loads are issued together, their per-head dot
   // products reduced together (U-way interleaved butterflies), and the running
   // state rescaled once per step.
   constexpr int U = 4;
 #pragma unroll 1
-  for (int key0 = t.kbeg + warp; key0 < t.kend; key0 += W * U) {
+  for (int key0 = t.kbeg + warp; key0 < t.kstream; key0 += W * U) {
     float kv[U][E], vv[U][E];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int key = key0 + u * W;
-      const bool live = key < t.kend;
+      const bool live = key < t.kstream;
       const size_t base = (static_cast<size_t>(t.o0) + (live ? key : t.kbeg)) * rs +
                           static_cast<size_t>(t.g) * D + lane * E;
 #pragma unroll
@@ -898,16 +986,19 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
       float mx = m[h];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        sc[u] = (key0 + u * W < t.kend) ? sc[u] * a.scale_log2 : -INFINITY;
+        const int key = key0 + u * W;
+        sc[u] = (key < t.kstream) ? fmaf(sc[u], a.scale_log2, bias2(a, t, key)) : -INFINITY;
         mx = fmaxf(mx, sc[u]);
       }
-      const float al = exp2f(m[h] - mx);
+      // every logit so far may be -inf (a masking bias): keep exp2 away from -inf - -inf
+      const float mu = (mx == -INFINITY) ? 0.f : mx;
+      const float al = exp2f(m[h] - mu);
       float lsum = l[h] * al;
 #pragma unroll
       for (int e = 0; e < E; ++e) o[h][e] *= al;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const float p = exp2f(sc[u] - mx);
+        const float p = exp2f(sc[u] - mu);
         lsum += p;
 #pragma unroll
         for (int e = 0; e < E; ++e) o[h][e] = fmaf(p, vv[u][e], o[h][e]);
@@ -916,9 +1007,11 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
       m[h] = mx;
     }
   }
+  // slots: W warps, plus the appended key when this tile owns it
   float* ms = fsm;
-  float* ls = ms + W * HP;
-  float* accs = ls + W * HP;
+  float* ls = ms + (W + 1) * HP;
+  float* accs = ls + (W + 1) * HP;
+  const int nslots = W + (t.append ? 1 : 0);
   if (lane == 0) {
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
@@ -926,19 +1019,31 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
       ls[warp * HP + h] = l[h];
     }
   }
+  if (t.append)
+    for (int h = threadIdx.x; h < HP; h += C::kThreads) {
+      ms[W * HP + h] = h < a.hpk ? smN[h] : -INFINITY;
+      ls[W * HP + h] = h < a.hpk ? 1.f : 0.f;
+    }
   __syncthreads();
 #pragma unroll
   for (int h = 0; h < HMAX; ++h) {
     if (h >= a.hpk) break;
     float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < W; ++w) M = fmaxf(M, ms[w * HP + h]);
+    for (int w = 0; w < nslots; ++w) M = fmaxf(M, ms[w * HP + h]);
     const float f = exp2f(m[h] - ((M == -INFINITY) ? 0.f : M));
 #pragma unroll
     for (int e = 0; e < E; ++e) accs[(warp * HP + h) * P + lane * E + e] = o[h][e] * f;
   }
+  if (t.append)
+    for (int i = threadIdx.x; i < a.hpk * D; i += C::kThreads) {
+      const int h = i / D, d = i % D;
+      float M = -INFINITY;
+      for (int w = 0; w < nslots; ++w) M = fmaxf(M, ms[w * HP + h]);
+      const float vn = static_cast<const float*>(a.v_new)[(static_cast<size_t>(t.b) * a.G + t.g) * D + d];
+      accs[(W * HP + h) * P + d] = vn * exp2f(ms[W * HP + h] - (M == -INFINITY ? 0.f : M));
+    }
   __syncthreads();
-  store_partial<D, W, HP>(a, t, ms, ls, accs, threadIdx.x, C::kThreads);
+  store_partial<D, W, HP>(a, t, ms, ls, accs, threadIdx.x, C::kThreads, nslots);
   if (a.merge) {
     __syncthreads();                         // store_partial done with the scratch
     finish_segment<D, HMAX>(a, t, threadIdx.x, smM, smL, smC, &smFlag, fsm, C::kWeightCap, 0u,
@@ -1041,6 +1146,33 @@ __global__ void __launch_bounds__(128) gqa_merge_kernel(const MergeArgs a) {
   if (threadIdx.x == 0 && a.om) {
     a.om[r] = (Lt == 0.f) ? -INFINITY : M;
     a.ol[r] = Lt;
+  }
+}
+
+// ============================================================================
+// index rows -> additive bias (metrale glm5next_dsa_ref, topk_to_mask)
+// ============================================================================
+
+// One CTA per sequence b: rows offsets[b]..offsets[b+1]-1 of `bias` become -inf,
+// then 0 at every in-range position named by idx[b, 0..width) (relative to the
+// sequence; -1 is the INVALID sentinel, repeats collapse, out-of-range entries
+// are dropped). Rows outside every sequence are not touched. Malformed offsets
+// leave the sequence alone and flag kErrBadOffsets.
+__global__ void __launch_bounds__(256) gqa_topk_to_bias_kernel(const int32_t* idx, int32_t width,
+                                                               const int32_t* offsets, int32_t max_len,
+                                                               float* bias, uint32_t* err) {
+  const int b = blockIdx.x;
+  const int o0 = offsets[b], o1 = offsets[b + 1];
+  if (!(0 <= o0 && o0 <= o1 && o1 <= max_len)) {
+    if (threadIdx.x == 0 && err) atomicOr(err, kErrBadOffsets);
+    return;
+  }
+  for (int r = o0 + threadIdx.x; r < o1; r += blockDim.x) bias[r] = -INFINITY;
+  __syncthreads();
+  const int n = o1 - o0;
+  for (int w = threadIdx.x; w < width; w += blockDim.x) {
+    const int t = idx[static_cast<size_t>(b) * width + w];
+    if (t >= 0 && t < n) bias[o0 + t] = 0.f;
   }
 }
 

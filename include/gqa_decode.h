@@ -128,6 +128,10 @@ typedef struct {
    * initialised once with gqa_workspace_init. Not shared by calls that overlap. */
   void* workspace;
   size_t workspace_bytes;
+  /* Optional additive logit bias, fp32 [max_len], one value per cache row, added
+   * to scale*q.k of that row for every query head ([attn.rs] self_attn_incremental
+   * `attn_bias`); -inf masks the key out. NULL = no bias. 4-byte aligned. */
+  const float* bias;
 } gqa_decode_params;
 
 /* Bytes of workspace gqa_decode_attend needs for these params, and the
@@ -176,6 +180,32 @@ gqa_status gqa_decode_attend(const gqa_decode_params* params, gqa_stream_t strea
  *     readable through gqa_get_device_error; use gqa_decode_attend with a
  *     workspace to diagnose malformed offsets. */
 gqa_status gqa_decode_attend_static_workspace(const gqa_decode_params* params, gqa_stream_t stream);
+
+/* One decode step with the new token appended first ([attn.rs]
+ * KvCache::push_kv, then self_attn_incremental): for every sequence b, cache row
+ * offsets[b+1]-1 -- the caller's offsets already count the new token -- receives
+ * k_new[b] and v_new[b] ([batch, num_kv_heads, head_dim], kv dtype, device,
+ * 16-byte aligned), and the attention covers offsets[b]..offsets[b+1]-1 with the
+ * new key included. params->k and params->v are WRITTEN (that one row per
+ * sequence and KV head). A sequence with no row (offsets[b] == offsets[b+1]) has
+ * no place for its token: it is skipped and GQA_ERR_BAD_OFFSETS is flagged in
+ * the device error word (the pages' push_kv drops a token when the cache is
+ * full). Everything else is as gqa_decode_attend. */
+gqa_status gqa_decode_append_attend(const gqa_decode_params* params, const void* k_new,
+                                    const void* v_new, gqa_stream_t stream);
+
+/* Index-selected attention as an additive bias (metrale glm5next_dsa_ref,
+ * `topk_to_mask`: the attention reads a mask built from an index row; repeated
+ * indices collapse, the INVALID sentinel -1 and out-of-range entries drop).
+ *   idx      device int32 [batch, width]: key positions relative to sequence b
+ *   offsets  device int32 [batch + 1], as for gqa_decode_attend
+ *   bias     device fp32 [max_len]: rows of every sequence become -inf except
+ *            the selected ones, which become 0; other rows are not touched
+ *   workspace  NULL, or a workspace whose error word takes GQA_ERR_BAD_OFFSETS
+ * Pass the result as gqa_decode_params.bias. width may be 0 (everything masked). */
+gqa_status gqa_topk_to_bias(const int32_t* idx, int32_t batch, int32_t width,
+                            const int32_t* offsets, int32_t max_len, float* bias,
+                            void* workspace, gqa_stream_t stream);
 
 /* Merge num_states states per row ([usearch] carry: partial-softmax rescaling):
  *   M = max m_i,  L = sum l_i e^{m_i - M},  ACC = sum acc_i e^{m_i - M}
