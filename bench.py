@@ -46,9 +46,16 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c2_bf16")
+    ap.add_argument("--op", choices=["attend", "append_attend", "masked_attend"], default="attend",
+                    help="attend: plain decode attention (the default line); append_attend: "
+                         "append the new token's K/V then attend; masked_attend: index rows -> "
+                         "bias (gqa_topk_to_bias) then attend with it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every step from Python instead of replaying a CUDA graph "
+                         "of the K steps")
     ap.add_argument("--quick", action="store_true",
                     help="timed loop and kernel timing only (no clock sampling, e2e or CPU "
                          "baseline); for profiler launch lists")
@@ -233,10 +240,34 @@ def run_ours(args):
     out = torch.empty(q.shape, dtype=q.dtype, device=dev)
     ws = gqa.Workspace(dev)
 
+    gen = torch.Generator().manual_seed(77)
+    k_new = torch.randn((w.batch, G, D), generator=gen).to(w.k.dtype).to(dev)
+    v_new = torch.randn((w.batch, G, D), generator=gen).to(w.k.dtype).to(dev)
+    width = 512
+    idx = torch.randint(-1, max(w.max_seq_len, 1), (w.batch, width), generator=gen,
+                        dtype=torch.int32).to(dev)
+    bias = torch.zeros(w.total_rows, dtype=torch.float32, device=dev)
+
     def step(i):
-        k, v = caches[i % len(caches)]
-        gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
-                              out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=stream)
+        run_op(*caches[i % len(caches)])
+
+    def step_on(i, st):
+        run_op(*caches[i % len(caches)], st)
+
+    def run_op(k, v, st=None):
+        st = st or stream
+        if args.op == "append_attend":
+            gqa.gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, H, G, score_scale=w.score_scale,
+                                         carry=carry, out=out, max_seq_len=w.max_seq_len, workspace=ws,
+                                         stream=st)
+        elif args.op == "masked_attend":
+            gqa.gqa_topk_to_bias(idx, offsets, w.total_rows, bias=bias, stream=st)
+            gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
+                                  out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st,
+                                  bias=bias)
+        else:
+            gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
+                                  out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st)
 
     def barrier():
         if world > 1:
@@ -247,6 +278,29 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert gqa.gqa_get_device_error(ws) == 0
 
+    # The timed K steps are captured once into a CUDA graph (the calls allocate
+    # nothing and never synchronise, so they capture as-is) and replayed: the
+    # host's per-call marshalling is then off the critical path, as in a serving
+    # loop. --eager launches them one by one instead.
+    graph = None
+    if not args.eager:
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap_stream = torch.cuda.current_stream()
+            for i in range(args.steps):
+                step_on(i, cap_stream)
+        torch.cuda.synchronize()
+        graph.replay()                   # one untimed replay
+        torch.cuda.synchronize()
+
+    def timed_steps():
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                step(i)
+
     sampler = ClockSampler(local) if not args.quick else None
     if sampler:
         sampler.start()
@@ -255,8 +309,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for i in range(args.steps):
-        step(i)
+    timed_steps()
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -265,9 +318,7 @@ def run_ours(args):
     extra_t0 = time.perf_counter()
     i = 0
     while sampler and ms_total / 1e3 + (time.perf_counter() - extra_t0) < 1.5:
-        for _ in range(200):
-            step(i)
-            i += 1
+        timed_steps()
         torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
 
@@ -319,8 +370,7 @@ def run_ours(args):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         offsets.copy_(hoff, non_blocking=True)
-        gqa.gqa_decode_attend(q, dk, dv, offsets, H, G, score_scale=w.score_scale, carry=carry, out=out,
-                              max_seq_len=w.max_seq_len, workspace=ws, stream=stream)
+        run_op(dk, dv)
         hout.copy_(out, non_blocking=True)
 
     n_e2e = 0 if args.quick else args.e2e_steps
@@ -358,7 +408,7 @@ def run_ours(args):
             "dtype": "bf16" if w.k.dtype == torch.bfloat16 else "f32",
             "data": "synthetic (seeded, no dataset)",
             "config": {
-                "workload": w.name, "text": w.meta.get("text", ""), "batch": w.batch,
+                "workload": w.name, "op": args.op, "text": w.meta.get("text", ""), "batch": w.batch,
                 "num_heads": H, "num_kv_heads": G, "head_dim": D, "seq_len": w.max_seq_len,
                 "kv_bytes_per_step": kv_bytes, "num_splits": S, "chunk_len": chunk,
                 "l2": f"inputs larger than L2: {len(caches)} cache copies of {kv_bytes / 2**20:.0f} MiB alternated",
@@ -379,7 +429,8 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * (2 if args.op == "masked_attend" else 1),
+            "launch_mode": "eager" if args.eager else "cuda_graph_of_timed_steps",
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
