@@ -21,6 +21,7 @@ import os
 __all__ = [
     "GqaError", "LibraryMissing", "State", "Workspace", "gqa_decode_attend",
     "gqa_decode_append_attend", "gqa_topk_to_bias", "gqa_decode_attend_static_workspace",
+    "gqa_softmax_merge_gathered",
     "gqa_decode_workspace_size", "gqa_workspace_init", "gqa_softmax_merge", "gqa_state_finalize",
     "gqa_get_device_error", "gqa_plan_splits", "gqa_status_string", "gqa_version", "lib_path",
     "load_library",
@@ -99,6 +100,7 @@ def load_library(path=None):
     lib.gqa_decode_append_attend.argtypes = [ctypes.POINTER(_CParams), sp, sp, sp]
     lib.gqa_topk_to_bias.argtypes = [sp, i32, i32, sp, i32, sp, sp, sp]
     lib.gqa_softmax_merge.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
+    lib.gqa_softmax_merge_gathered.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
     lib.gqa_state_finalize.argtypes = [ps, i32, i32, sp, i32, sp]
     lib.gqa_get_device_error.argtypes = [sp, sp]
     lib.gqa_plan_splits.argtypes = [i32, i32, i32, i64, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
@@ -107,7 +109,7 @@ def load_library(path=None):
     lib.gqa_version.argtypes = []
     for fn in ("gqa_decode_workspace_size", "gqa_workspace_init", "gqa_decode_attend", "gqa_softmax_merge",
                "gqa_state_finalize", "gqa_get_device_error", "gqa_plan_splits",
-               "gqa_decode_append_attend", "gqa_topk_to_bias"):
+               "gqa_decode_append_attend", "gqa_topk_to_bias", "gqa_softmax_merge_gathered"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gqa_version.restype = ctypes.c_int32
     if path is None:
@@ -365,6 +367,28 @@ def gqa_softmax_merge(states, carry=None, merged_out=None, out=None, out_dtype=N
     _check(load_library().gqa_softmax_merge(ctypes.byref(cs), rows, S, D, ctypes.byref(cc),
                                             ctypes.byref(cm), _ptr(out), odt, _stream_handle(stream)),
            "gqa_softmax_merge")
+    return out
+
+
+def gqa_softmax_merge_gathered(states, carry=None, merged_out=None, out=None, out_dtype=None,
+                               want_out=None, stream=None):
+    """Merge states gathered as m, l [S, rows]; acc [S, rows, D] (one block per
+    contributor, as an all-gather lays them out) with an optional carry."""
+    torch = _torch()
+    S, rows = states.m.shape
+    D = states.acc.shape[-1]
+    if want_out is None:
+        want_out = out is not None or merged_out is None
+    if want_out and out is None:
+        out = torch.empty((rows, D), dtype=out_dtype or torch.float32, device=states.m.device)
+    odt = _dtype_code(out) if out is not None else GQA_F32
+    cs = states._c()
+    cc = _c_state(carry)
+    cm = _c_state(merged_out)
+    _check(load_library().gqa_softmax_merge_gathered(ctypes.byref(cs), rows, S, D, ctypes.byref(cc),
+                                                     ctypes.byref(cm), _ptr(out), odt,
+                                                     _stream_handle(stream)),
+           "gqa_softmax_merge_gathered")
     return out
 
 

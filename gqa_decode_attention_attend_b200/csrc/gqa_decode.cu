@@ -532,7 +532,7 @@ gqa_status gqa_topk_to_bias(const int32_t* idx, int32_t batch, int32_t width, co
 
 static gqa_status merge_common(const gqa_state* states, int32_t rows, int32_t num_states, int32_t head_dim,
                                const gqa_state* carry_in, const gqa_state* merged_out, void* out,
-                               int32_t out_dtype, gqa_stream_t stream) {
+                               int32_t out_dtype, gqa_stream_t stream, bool gathered = false) {
   if (rows < 0 || num_states < 0 || (head_dim != 64 && head_dim != 128)) return GQA_ERR_INVALID_ARGUMENT;
   if (num_states > 0 && (!states || !state_complete(*states))) return GQA_ERR_INVALID_ARGUMENT;
   const bool has_carry = carry_in && state_present(*carry_in);
@@ -561,6 +561,8 @@ static gqa_status merge_common(const gqa_state* states, int32_t rows, int32_t nu
   m.acc = num_states > 0 ? states->acc : nullptr;
   m.rows = rows;
   m.S = num_states;
+  m.row_stride = gathered ? 1 : num_states;
+  m.state_stride = gathered ? rows : 1;
   m.cm = has_carry ? carry_in->m : nullptr;
   m.cl = has_carry ? carry_in->l : nullptr;
   m.cacc = has_carry ? carry_in->acc : nullptr;
@@ -578,6 +580,13 @@ gqa_status gqa_softmax_merge(const gqa_state* states, int32_t rows, int32_t num_
                              const gqa_state* carry_in, const gqa_state* merged_out, void* out,
                              int32_t out_dtype, gqa_stream_t stream) {
   return merge_common(states, rows, num_states, head_dim, carry_in, merged_out, out, out_dtype, stream);
+}
+
+gqa_status gqa_softmax_merge_gathered(const gqa_state* states, int32_t rows, int32_t num_states,
+                                      int32_t head_dim, const gqa_state* carry_in,
+                                      const gqa_state* merged_out, void* out, int32_t out_dtype,
+                                      gqa_stream_t stream) {
+  return merge_common(states, rows, num_states, head_dim, carry_in, merged_out, out, out_dtype, stream, true);
 }
 
 gqa_status gqa_state_finalize(const gqa_state* state, int32_t rows, int32_t head_dim, void* out,

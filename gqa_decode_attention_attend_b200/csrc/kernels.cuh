@@ -1056,10 +1056,12 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
 // ============================================================================
 
 struct MergeArgs {
-  const float* m;            // [rows, S]
-  const float* l;            // [rows, S]
-  const float* acc;          // [rows, S, D]
+  const float* m;            // state (r, i) at r * row_stride + i * state_stride
+  const float* l;
+  const float* acc;          // ... times D
   int32_t rows, S;
+  int64_t row_stride;        // S for [rows, S] (split-major), 1 for [S, rows] (gathered)
+  int64_t state_stride;      // 1 for [rows, S], rows for [S, rows]
   const float* cm;           // carry [rows] / [rows, D], or null
   const float* cl;
   const float* cacc;
@@ -1079,11 +1081,12 @@ __global__ void __launch_bounds__(128) gqa_merge_kernel(const MergeArgs a) {
   const int r = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nS = a.S;
-  const size_t base = static_cast<size_t>(r) * a.S;
+  const size_t base = static_cast<size_t>(r) * a.row_stride;
+  const size_t ss = static_cast<size_t>(a.state_stride);
   // pass 1: the largest maximum among non-empty states (and the carry)
   float M = -INFINITY;
   for (int i = threadIdx.x; i < nS; i += blockDim.x)
-    if (a.l[base + i] != 0.f) M = fmaxf(M, a.m[base + i]);
+    if (a.l[base + i * ss] != 0.f) M = fmaxf(M, a.m[base + i * ss]);
   for (int x = 16; x >= 1; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
   if (lane == 0) red[warp] = M;
   __syncthreads();
@@ -1103,11 +1106,11 @@ __global__ void __launch_bounds__(128) gqa_merge_kernel(const MergeArgs a) {
   if (M != -INFINITY) {
 #pragma unroll 4
     for (int i = warp; i < nS; i += W) {
-      const float li = a.l[base + i];
+      const float li = a.l[base + i * ss];
       if (li == 0.f) continue;
-      const float w = expf(a.m[base + i] - M);
+      const float w = expf(a.m[base + i * ss] - M);
       L += li * w;
-      const float* src = a.acc + (base + i) * D + lane * E;
+      const float* src = a.acc + (base + i * ss) * D + lane * E;
       if constexpr (E == 4) {
         const float4 v = *reinterpret_cast<const float4*>(src);
         acc[0] = fmaf(v.x, w, acc[0]);

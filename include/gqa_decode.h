@@ -220,6 +220,17 @@ gqa_status gqa_softmax_merge(const gqa_state* states, int32_t rows, int32_t num_
                              const gqa_state* merged_out, void* out, int32_t out_dtype,
                              gqa_stream_t stream);
 
+/* The same merge for states laid out [num_states, rows] (m, l) and
+ * [num_states, rows, head_dim] (acc) -- one block per contributor, the layout an
+ * all-gather of per-rank states produces (context-parallel decode: each rank
+ * attends over its slice of every sequence's keys, the states are exchanged,
+ * and this merge folds them with the carry). Arguments otherwise as
+ * gqa_softmax_merge. */
+gqa_status gqa_softmax_merge_gathered(const gqa_state* states, int32_t rows, int32_t num_states,
+                                      int32_t head_dim, const gqa_state* carry_in,
+                                      const gqa_state* merged_out, void* out, int32_t out_dtype,
+                                      gqa_stream_t stream);
+
 /* out = acc / l per row (0 when l == 0), cast to out_dtype ([usearch]: outputs
  * land already divided by the partition). state [rows], out [rows, head_dim]. */
 gqa_status gqa_state_finalize(const gqa_state* state, int32_t rows, int32_t head_dim, void* out,
