@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-early-start", action="store_true",
+                    help="launch every call in plain stream order instead of with "
+                         "GQA_FLAG_EARLY_START (steps here never write the cache rows or "
+                         "offsets the next step reads, which is that flag's contract)")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step from Python instead of replaying a CUDA graph "
                          "of the K steps")
@@ -254,20 +258,22 @@ def run_ours(args):
     def step_on(i, st):
         run_op(*caches[i % len(caches)], st)
 
+    flags = 0 if args.no_early_start else gqa.GQA_FLAG_EARLY_START
+
     def run_op(k, v, st=None):
         st = st or stream
         if args.op == "append_attend":
             gqa.gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, H, G, score_scale=w.score_scale,
                                          carry=carry, out=out, max_seq_len=w.max_seq_len, workspace=ws,
-                                         stream=st)
+                                         stream=st, flags=flags)
         elif args.op == "masked_attend":
-            gqa.gqa_topk_to_bias(idx, offsets, w.total_rows, bias=bias, stream=st)
+            gqa.gqa_topk_to_bias(idx, offsets, w.total_rows, bias=bias, stream=st, flags=flags)
             gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
                                   out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st,
-                                  bias=bias)
+                                  bias=bias, flags=flags)
         else:
             gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
-                                  out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st)
+                                  out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st, flags=flags)
 
     def barrier():
         if world > 1:
@@ -430,7 +436,8 @@ def run_ours(args):
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * (2 if args.op == "masked_attend" else 1),
-            "launch_mode": "eager" if args.eager else "cuda_graph_of_timed_steps",
+            "launch_mode": ("eager" if args.eager else "cuda_graph_of_timed_steps") +
+                           ("" if args.no_early_start else "+early_start"),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

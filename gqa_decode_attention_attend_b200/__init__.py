@@ -39,6 +39,7 @@ GQA_ERR_BAD_OFFSETS = 5
 GQA_ERR_TIMEOUT = 6
 GQA_F32 = 0
 GQA_BF16 = 1
+GQA_FLAG_EARLY_START = 1
 
 
 class LibraryMissing(RuntimeError):
@@ -70,6 +71,7 @@ class _CParams(ctypes.Structure):
         ("num_splits", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("bias", ctypes.c_void_p),
+        ("flags", ctypes.c_uint32),
     ]
 
 
@@ -228,7 +230,7 @@ def _default_workspace(device):
 
 
 def _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out,
-            out_dtype, partials_out, num_splits, max_seq_len, max_len, bias=None):
+            out_dtype, partials_out, num_splits, max_seq_len, max_len, bias=None, flags=0):
     p = _CParams()
     p.struct_size = ctypes.sizeof(_CParams)
     p.q, p.q_dtype = _ptr(q), _dtype_code(q)
@@ -254,6 +256,7 @@ def _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state
         if bias.dtype != torch.float32:
             raise GqaError(GQA_ERR_SHAPE_MISMATCH, "bias must be float32")
     p.bias = _ptr(bias)
+    p.flags = int(flags)
     return p
 
 
@@ -277,7 +280,7 @@ def gqa_decode_workspace_size(q, k, v, offsets, num_heads, num_kv_heads=0, *, sc
 
 def _attend_call(entry, q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out,
                  out_dtype, partials_out, want_out, num_splits, max_seq_len, max_len, workspace, stream,
-                 bias, extra=()):
+                 bias, extra=(), flags=0):
     torch = _torch()
     if want_out is None:
         want_out = out is not None or (state_out is None and partials_out is None)
@@ -288,7 +291,7 @@ def _attend_call(entry, q, k, v, offsets, num_heads, num_kv_heads, score_scale, 
     if out is not None:
         odt = _dtype_code(out)
     p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
-                partials_out, num_splits, max_seq_len, max_len, bias)
+                partials_out, num_splits, max_seq_len, max_len, bias, flags)
     lib = load_library()
     nbytes = ctypes.c_size_t()
     _check(lib.gqa_decode_workspace_size(ctypes.byref(p), ctypes.byref(nbytes), None, None),
@@ -304,7 +307,7 @@ def _attend_call(entry, q, k, v, offsets, num_heads, num_kv_heads, score_scale, 
 def gqa_decode_attend(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scale=0.0, carry=None,
                       state_out=None, out=None, out_dtype=None, partials_out=None, want_out=None,
                       num_splits=0, max_seq_len=0, max_len=None, workspace=None, stream=None,
-                      bias=None):
+                      bias=None, flags=0):
     """Decode attention over a KV cache; see include/gqa_decode.h.
 
     q [B, H, D]; k, v [max_len, G, D]; offsets int32 [B+1] on the device.
@@ -315,13 +318,13 @@ def gqa_decode_attend(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scal
     """
     return _attend_call("gqa_decode_attend", q, k, v, offsets, num_heads, num_kv_heads, score_scale,
                         carry, state_out, out, out_dtype, partials_out, want_out, num_splits,
-                        max_seq_len, max_len, workspace, stream, bias)
+                        max_seq_len, max_len, workspace, stream, bias, flags=flags)
 
 
 def gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_heads=0, *,
                              score_scale=0.0, carry=None, state_out=None, out=None, out_dtype=None,
                              want_out=None, num_splits=0, max_seq_len=0, max_len=None,
-                             workspace=None, stream=None, bias=None):
+                             workspace=None, stream=None, bias=None, flags=0):
     """Append k_new/v_new [B, G, D] at row offsets[b+1]-1 of the caches (which
     are written), then attend with the new key included; see include/gqa_decode.h."""
     if k_new.dtype != k.dtype or v_new.dtype != k.dtype:
@@ -329,7 +332,7 @@ def gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_h
     return _attend_call("gqa_decode_append_attend", q, k, v, offsets, num_heads, num_kv_heads,
                         score_scale, carry, state_out, out, out_dtype, None, want_out, num_splits,
                         max_seq_len, max_len, workspace, stream, bias,
-                        extra=(ctypes.c_void_p(_ptr(k_new)), ctypes.c_void_p(_ptr(v_new))))
+                        extra=(ctypes.c_void_p(_ptr(k_new)), ctypes.c_void_p(_ptr(v_new))), flags=flags)
 
 
 def gqa_topk_to_bias(idx, offsets, max_len, bias=None, workspace=None, stream=None):

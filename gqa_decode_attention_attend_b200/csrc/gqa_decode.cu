@@ -270,6 +270,7 @@ gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
   if (align_or & 15u) return GQA_ERR_SHAPE_MISMATCH;
   if (reinterpret_cast<uintptr_t>(p->bias) & 3u) return GQA_ERR_SHAPE_MISMATCH;
   if (!std::isfinite(p->score_scale)) return GQA_ERR_INVALID_ARGUMENT;
+  if (p->flags & ~static_cast<uint32_t>(GQA_FLAG_EARLY_START)) return GQA_ERR_INVALID_ARGUMENT;
   r->scale = p->score_scale != 0.f ? p->score_scale : 1.0f / sqrtf(static_cast<float>(r->D));
   if (static_cast<int64_t>(r->B) * r->H * r->D > INT32_MAX) return GQA_ERR_INVALID_ARGUMENT;
 
@@ -335,38 +336,58 @@ cudaError_t launch_merge_any(int D, const MergeArgs& m, cudaStream_t st) {
   return D == 128 ? launch_merge<128>(m, st) : launch_merge<64>(m, st);
 }
 
+// Launch configuration shared by the partition kernels. With early_start the
+// launch carries programmatic stream serialization: the kernel may begin while
+// the previous kernel on the stream finishes (see GQA_FLAG_EARLY_START).
+struct Launch {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  Launch(unsigned grid, unsigned threads, size_t smem, cudaStream_t st, bool early_start) {
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = early_start ? 1 : 0;
+  }
+};
+
 template <int D, int NT>
 cudaError_t launch_bf16(const PartitionArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                        unsigned grid, cudaStream_t st) {
+                        unsigned grid, cudaStream_t st, bool early) {
   using C = gqa::TcCfg<D, NT>;
-  gqa::gqa_partition_bf16_kernel<D, NT><<<grid, C::kThreads, C::kSmemBytes, st>>>(tk, tv, a);
-  return cudaGetLastError();
+  Launch l(grid, C::kThreads, C::kSmemBytes, st, early);
+  return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_bf16_kernel<D, NT>, tk, tv, a);
 }
 
 template <int D, int HMAX>
-cudaError_t launch_f32(const PartitionArgs& a, unsigned grid, cudaStream_t st) {
+cudaError_t launch_f32(const PartitionArgs& a, unsigned grid, cudaStream_t st, bool early) {
   using C = gqa::F32Cfg<D, HMAX>;
-  gqa::gqa_partition_f32_kernel<D, HMAX><<<grid, C::kThreads, C::kSmemBytes, st>>>(a);
-  return cudaGetLastError();
+  Launch l(grid, C::kThreads, C::kSmemBytes, st, early);
+  return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_f32_kernel<D, HMAX>, a);
 }
 
 cudaError_t launch_partition(const Resolved& r, const PartitionArgs& a, const CUtensorMap* tk,
-                             const CUtensorMap* tv, cudaStream_t st) {
+                             const CUtensorMap* tv, cudaStream_t st, bool early) {
   const unsigned grid = static_cast<unsigned>(r.B) * r.S * r.G;
   if (grid == 0) return cudaSuccess;
   if (r.bf16) {
     const int nt = nt_of(r.hpk);
-    if (r.D == 128) return nt == 1 ? launch_bf16<128, 1>(a, *tk, *tv, grid, st) : launch_bf16<128, 2>(a, *tk, *tv, grid, st);
-    return nt == 1 ? launch_bf16<64, 1>(a, *tk, *tv, grid, st) : launch_bf16<64, 2>(a, *tk, *tv, grid, st);
+    if (r.D == 128)
+      return nt == 1 ? launch_bf16<128, 1>(a, *tk, *tv, grid, st, early) : launch_bf16<128, 2>(a, *tk, *tv, grid, st, early);
+    return nt == 1 ? launch_bf16<64, 1>(a, *tk, *tv, grid, st, early) : launch_bf16<64, 2>(a, *tk, *tv, grid, st, early);
   }
   if (r.D == 128) {
-    if (r.hpk <= 4) return launch_f32<128, 4>(a, grid, st);
-    if (r.hpk <= 8) return launch_f32<128, 8>(a, grid, st);
-    return launch_f32<128, 16>(a, grid, st);
+    if (r.hpk <= 4) return launch_f32<128, 4>(a, grid, st, early);
+    if (r.hpk <= 8) return launch_f32<128, 8>(a, grid, st, early);
+    return launch_f32<128, 16>(a, grid, st, early);
   }
-  if (r.hpk <= 4) return launch_f32<64, 4>(a, grid, st);
-  if (r.hpk <= 8) return launch_f32<64, 8>(a, grid, st);
-  return launch_f32<64, 16>(a, grid, st);
+  if (r.hpk <= 4) return launch_f32<64, 4>(a, grid, st, early);
+  if (r.hpk <= 8) return launch_f32<64, 8>(a, grid, st, early);
+  return launch_f32<64, 16>(a, grid, st, early);
 }
 
 // Pointer checks and the single launch of a decode call, with the scratch at `ws`
@@ -440,7 +461,10 @@ gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* w
     cudaGetLastError();
     return GQA_ERR_DEVICE;
   }
-  if (launch_partition(r, a, &tk, &tv, cs) != cudaSuccess) return GQA_ERR_DEVICE;
+  if (launch_partition(r, a, &tk, &tv, cs, (p->flags & GQA_FLAG_EARLY_START) != 0) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
   return GQA_OK;
 }
 

@@ -597,6 +597,7 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
 
   const Tile t = tile_of(a, blockIdx.x);
   if (t.kbeg >= t.kend) {
+    ptx::grid_dependency_wait();
     if (a.write_empty) write_empty_states<D>(a, t);
     // A sequence without keys: split 0 still writes its rows (carry or zeros).
     if (a.merge && t.n == 0 && t.c == 0 && warp < C::kConsumerWarps)
@@ -656,6 +657,10 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 
   // ------------------------------------------------------------ consumer warps
+  // Everything the previous kernel on the stream may have written (q, carry,
+  // bias, the appended K/V, the workspace) is read only after this wait; the
+  // producer's cache loads above may run ahead of it (early-start launches).
+  ptx::grid_dependency_wait();
   // Q^T as the B operand of S^T = K Q^T: b0 = q[head][k0 + 2*(lane%4) + {0,1}],
   // b1 = the same 8 columns further, head = nt*8 + lane/4 (zero past hpk).
   uint32_t qf[D / 16][NT][2];
@@ -818,6 +823,10 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 
   // ------------------------------------------------------------ epilogue
+  // The tile's cache stream is done: the next kernel on the stream may now be
+  // scheduled (it still waits for this grid before reading what it writes), so
+  // its first loads overlap this grid's epilogue and merges.
+  if (threadIdx.x == 0) ptx::grid_launch_dependents();
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -917,6 +926,7 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
   __shared__ float smM[16], smL[16], smC[16], smN[16];
   __shared__ int smFlag;
   const Tile t = tile_of(a, blockIdx.x);
+  ptx::grid_dependency_wait();
   if (t.kbeg >= t.kend) {
     if (a.write_empty) write_empty_states<D>(a, t);
     if (a.merge && t.n == 0 && t.c == 0)
@@ -1007,6 +1017,7 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
       m[h] = mx;
     }
   }
+  if (threadIdx.x == 0) ptx::grid_launch_dependents();   // cache stream done (see the bf16 kernel)
   // slots: W warps, plus the appended key when this tile owns it
   float* ms = fsm;
   float* ls = ms + (W + 1) * HP;

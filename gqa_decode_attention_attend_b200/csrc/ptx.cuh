@@ -123,6 +123,22 @@ __device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* addr, uint3
   return old;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Block until the grid this one depends on (the previous kernel on the stream,
+// when launched with programmatic stream serialization) has completed and its
+// memory is visible; returns at once when there is no such dependency.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next grid on the stream be scheduled once every CTA of this grid has
+// issued this (or exited); that grid still waits for this one before it reads
+// what this one writes.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- named barriers
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {

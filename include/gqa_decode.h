@@ -69,6 +69,17 @@ typedef enum {
 
 typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
 
+/* Flags of gqa_decode_params.flags.
+ * GQA_FLAG_EARLY_START: launch with programmatic stream serialization, so the
+ *   call's kernel may start -- and begin streaming K/V cache rows -- while the
+ *   kernel before it on the stream is still finishing. Everything else that
+ *   kernel may write (q, the carry, the bias, the appended K/V, the workspace)
+ *   is read only after it completes. The caller promises that the kernel
+ *   immediately before this call does not write the offsets or any cache row
+ *   this call reads from the cache (the row an append call writes itself is
+ *   not read from the cache). Without the flag, ordinary stream order. */
+enum { GQA_FLAG_EARLY_START = 1u };
+
 /* An online-softmax state per query row, structure of arrays, fp32 device memory:
  *   m   [rows]        running maximum of the logits scale*q.k, natural-log units
  *                     ([usearch] DenseSoftmaxState::maximum_score)
@@ -132,6 +143,7 @@ typedef struct {
    * to scale*q.k of that row for every query head ([attn.rs] self_attn_incremental
    * `attn_bias`); -inf masks the key out. NULL = no bias. 4-byte aligned. */
   const float* bias;
+  uint32_t flags;            /* GQA_FLAG_* bits; 0 = none */
 } gqa_decode_params;
 
 /* Bytes of workspace gqa_decode_attend needs for these params, and the

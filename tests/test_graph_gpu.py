@@ -57,3 +57,42 @@ def test_captured_append_step():
     graph.replay()
     torch.cuda.synchronize()
     assert torch.equal(out, eager)
+
+
+@pytest.mark.parametrize("graph", [False, True], ids=["eager", "graph"])
+def test_early_start_respects_a_carry_chain(graph):
+    """Three calls where each folds the previous one's state as its carry: with
+    GQA_FLAG_EARLY_START the kernel may start early, but it must read the carry
+    only after the previous kernel is done, so the chain matches plain order."""
+    dev = gu.device()
+    w = workloads.make("chain", [5000, 300, 64], 32, 8, 128, seed=23)
+    dw = gu.DevWorkload(w, dev)
+    rows = w.batch * w.num_heads
+    ws = gqa.Workspace(dev, 1 << 20)
+
+    def chain(flags, states, out):
+        carry = None
+        for st in states:
+            gqa.gqa_decode_attend(dw.q, dw.k, dw.v, dw.offsets, 32, 8, carry=carry, state_out=st,
+                                  want_out=False, workspace=ws, max_seq_len=5000, flags=flags)
+            carry = st
+        gqa.gqa_decode_attend(dw.q, dw.k, dw.v, dw.offsets, 32, 8, carry=carry, out=out,
+                              workspace=ws, max_seq_len=5000, flags=flags)
+
+    ref_states = [gqa.State.empty(rows, 128, dev) for _ in range(3)]
+    ref = torch.empty_like(dw.q)
+    chain(0, ref_states, ref)
+    torch.cuda.synchronize()
+    states = [gqa.State.empty(rows, 128, dev) for _ in range(3)]
+    out = torch.empty_like(dw.q)
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            chain(gqa.GQA_FLAG_EARLY_START, states, out)
+        g.replay()
+    else:
+        chain(gqa.GQA_FLAG_EARLY_START, states, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    for a, b in zip(states, ref_states):
+        assert torch.equal(a.acc, b.acc) and torch.equal(a.l, b.l)
