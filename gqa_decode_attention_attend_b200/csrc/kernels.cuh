@@ -646,6 +646,11 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         ++issued;
       }
+      // Every load of the tile is issued (its last stages are in flight): the
+      // next kernel on the stream may now be scheduled. It still waits for this
+      // grid before reading what it writes, so its first cache loads overlap
+      // this grid's last stages, epilogue and merges.
+      ptx::grid_launch_dependents();
       if (*abort_flag) {
         // Drain the copies still in flight before the CTA's shared memory goes away.
         for (int it = max(0, issued - C::kStages); it < issued; ++it)
@@ -823,10 +828,6 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 
   // ------------------------------------------------------------ epilogue
-  // The tile's cache stream is done: the next kernel on the stream may now be
-  // scheduled (it still waits for this grid before reading what it writes), so
-  // its first loads overlap this grid's epilogue and merges.
-  if (threadIdx.x == 0) ptx::grid_launch_dependents();
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll

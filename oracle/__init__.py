@@ -61,6 +61,11 @@ def load(path=None):
     lib.oracle_softmax_merge.argtypes = [
         _f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
         _f32p, _f32p, _f32p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+    lib.oracle_reconstruct_words.restype = ctypes.c_int
+    lib.oracle_reconstruct_words.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int64, ctypes.c_int,
+                                             _f32p, ctypes.c_int, ctypes.c_int, _f64p]
+    lib.oracle_f16_to_f64.restype = ctypes.c_double
+    lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_to_f64.restype = ctypes.c_double
     lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
     lib.oracle_default_threads.restype = ctypes.c_int
@@ -74,7 +79,8 @@ def _ptr(a, t):
 
 
 def _as_stored(x):
-    """Return (contiguous ndarray, is_bf16) for an fp32 array or bf16 bits.
+    """Return (contiguous ndarray, kind) for an fp32 array (0), bf16 bits (1)
+    or f64 (2, e.g. a reconstructed cache).
 
     bf16 data is passed as its raw uint16 bit patterns (numpy has no bf16).
     """
@@ -83,7 +89,9 @@ def _as_stored(x):
         return x, 1
     if x.dtype == np.float32:
         return x, 0
-    raise TypeError(f"oracle inputs are float32 or bf16 bits (uint16), got {x.dtype}")
+    if x.dtype == np.float64:
+        return x, 2
+    raise TypeError(f"oracle inputs are float32, f64 or bf16 bits (uint16), got {x.dtype}")
 
 
 class State:
@@ -196,6 +204,38 @@ def append_then_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_heads, 
     st = decode_attend(q, k2, v2, offsets.astype(np.int32), num_heads, num_kv_heads, score_scale,
                        **kw)
     return st, k2, v2
+
+
+def reconstruct_words(codes, atoms, lib=None):
+    """f64 rows from dictionary code words: codes uint32 [..., words] (atom index
+    in the high 16 bits, f16 coefficient bits in the low 16), atoms fp32
+    [n_atoms, D]. Returns f64 [..., D]."""
+    lib = lib or load()
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    atoms = np.ascontiguousarray(atoms, dtype=np.float32)
+    words = codes.shape[-1]
+    n = int(np.prod(codes.shape[:-1]))
+    D = atoms.shape[1]
+    out = np.empty((n, D), np.float64)
+    rc = lib.oracle_reconstruct_words(codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint32)), n, words,
+                                      _ptr(atoms, _f32p), atoms.shape[0], D, _ptr(out, _f64p))
+    if rc != 0:
+        raise ValueError("oracle_reconstruct_words refused its arguments")
+    return out.reshape(*codes.shape[:-1], D)
+
+
+def coded_decode_attend(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_heads, num_kv_heads,
+                        score_scale=0.0, lib=None, **kw):
+    """Decode attention over a dictionary-coded cache: reconstruct K and V
+    (f64, from the code words) and apply the plain definition."""
+    k = reconstruct_words(k_codes, k_atoms, lib=lib)
+    v = reconstruct_words(v_codes, v_atoms, lib=lib)
+    return decode_attend(q, k, v, offsets, num_heads, num_kv_heads, score_scale, lib=lib, **kw)
+
+
+def f16_to_f64(bits, lib=None):
+    lib = lib or load()
+    return lib.oracle_f16_to_f64(int(bits))
 
 
 def bf16_to_f64(bits, lib=None):

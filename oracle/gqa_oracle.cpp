@@ -65,8 +65,26 @@ inline double bf16_bits_to_f64(uint16_t bits) {
   return static_cast<double>(f);
 }
 
+// IEEE binary16 bits -> f64, from the format's definition (sign, 5-bit biased
+// exponent, 10-bit fraction; exponent 0 is subnormal, 31 is inf/NaN).
+inline double f16_bits_to_f64(uint16_t bits) {
+  const int sign = bits >> 15;
+  const int e = (bits >> 10) & 0x1F;
+  const int f = bits & 0x3FF;
+  double v;
+  if (e == 0)
+    v = std::ldexp(static_cast<double>(f), -24);
+  else if (e == 31)
+    v = f ? std::numeric_limits<double>::quiet_NaN() : std::numeric_limits<double>::infinity();
+  else
+    v = std::ldexp(static_cast<double>(1024 + f), e - 25);
+  return sign ? -v : v;
+}
+
+// Element of a stored array: kind 0 = fp32, 1 = bf16 bits, 2 = f64.
 inline double load_elem(const void* base, int is_bf16, int64_t idx) {
-  if (is_bf16) return bf16_bits_to_f64(static_cast<const uint16_t*>(base)[idx]);
+  if (is_bf16 == 1) return bf16_bits_to_f64(static_cast<const uint16_t*>(base)[idx]);
+  if (is_bf16 == 2) return static_cast<const double*>(base)[idx];
   return static_cast<double>(static_cast<const float*>(base)[idx]);
 }
 
@@ -321,6 +339,39 @@ int oracle_topk_to_bias(const int32_t* idx, int B, int width, const int32_t* off
   }
   return 0;
 }
+
+// Reconstruction of a dictionary-coded cache (qualiaDB KvDictionary:
+// `reconstruct_from_words`, the f16-coefficient inverse of `encode_to_words`;
+// `reconstruct`: sum of coeff * atom). Every cache row of every KV head is
+// `words` code words; word w holds the atom index in its high 16 bits and the
+// coefficient's IEEE binary16 bits in its low 16 bits (a zero coefficient,
+// as in padding words, reconstructs to nothing). atoms [n_atoms, D] fp32.
+// out [rows*G, D] f64: out_r = sum_w f16(coeff_w) * atoms[index_w].
+// Returns -1 if an index is out of range.
+int oracle_reconstruct_words(const uint32_t* codes, int64_t rows_x_heads, int words, const float* atoms,
+                             int n_atoms, int D, double* out) {
+  if (!codes || !atoms || !out || words <= 0 || n_atoms <= 0 || D <= 0) return -1;
+  for (int64_t r = 0; r < rows_x_heads; ++r) {
+    double* o = out + r * D;
+    for (int c = 0; c < D; ++c) o[c] = 0.0;
+    for (int w = 0; w < words; ++w) {
+      const uint32_t word = codes[r * words + w];
+#if ORACLE_MUTATION == 11
+      const int idx = static_cast<int>(word & 0xFFFF);              // fields swapped
+      const double coeff = f16_bits_to_f64(static_cast<uint16_t>(word >> 16));
+#else
+      const int idx = static_cast<int>(word >> 16);
+      const double coeff = f16_bits_to_f64(static_cast<uint16_t>(word & 0xFFFF));
+#endif
+      if (coeff == 0.0) continue;
+      if (idx >= n_atoms) return -1;
+      for (int c = 0; c < D; ++c) o[c] += coeff * static_cast<double>(atoms[static_cast<int64_t>(idx) * D + c]);
+    }
+  }
+  return 0;
+}
+
+double oracle_f16_to_f64(uint16_t bits) { return f16_bits_to_f64(bits); }
 
 // bf16 bits -> f64, exposed so the pins can check the widening on fixed patterns.
 double oracle_bf16_to_f64(uint16_t bits) { return bf16_bits_to_f64(bits); }

@@ -17,7 +17,10 @@ AssertionError when the oracle disagrees with:
   * the additive bias row -- brute force with the bias added after the scale; a
     constant bias only shifts m; a -inf bias equals removing the key; index rows
     turned into a mask keep exactly the distinct in-range indices; appending a
-    token writes only its row and attends over it.
+    token writes only its row and attends over it;
+  * the dictionary-coded cache -- binary16 coefficients on fixed bit patterns;
+    reconstruction against numpy's sum of coefficient * atom; one-hot codes
+    over the cache's own rows give plain attention exactly.
 
 Sources: needle_core ``attn.rs`` (``KvCache`` layout, ``self_attn_incremental``
 head map and scale); USearch linear algebra § Attention (online softmax folded
@@ -25,7 +28,8 @@ into the walk, carry by partial-softmax rescaling, outputs divided by the
 partition, ``score_scale`` zero derives it); cortiq_engine ``NystromState``
 example ``trial`` (planted key); metrale glm5next_dsa_ref ``pool_states``
 (empty softmax gives 0, not NaN) and ``topk_to_mask`` (index rows -> mask);
-needle_core ``attn.rs`` ``attn_bias`` and ``KvCache::push_kv``.
+needle_core ``attn.rs`` ``attn_bias`` and ``KvCache::push_kv``; qualiaDB
+``KvDictionary`` ``reconstruct`` / ``reconstruct_from_words``.
 """
 import math
 
@@ -53,6 +57,10 @@ class OracleHandle:
     def topk_to_bias(self, *a, **kw):
         kw.setdefault("lib", self.lib)
         return self.pkg.topk_to_bias(*a, **kw)
+
+    def reconstruct(self, *a, **kw):
+        kw.setdefault("lib", self.lib)
+        return self.pkg.reconstruct_words(*a, **kw)
 
 
 def _rng(seed):
@@ -404,11 +412,55 @@ def pin_append_then_attend(o):
     _close(st.out, brute_force(q, k2, v2, off, H, G, 1 / math.sqrt(D)), what="append then attend")
 
 
+def _pack(idx, coeff):
+    """Code word: atom index high 16 bits, coefficient's binary16 bits low 16."""
+    bits = np.asarray(coeff, np.float16).view(np.uint16).astype(np.uint32)
+    return (np.asarray(idx, np.uint32) << 16) | bits
+
+
+def pin_f16_coefficients(o):
+    cases = {0x3C00: 1.0, 0xC000: -2.0, 0x7BFF: 65504.0, 0x0001: 2.0 ** -24, 0x0400: 2.0 ** -14,
+             0x3555: 0.333251953125, 0x0000: 0.0, 0x8000: -0.0}
+    for bits, want in cases.items():
+        assert o.pkg.f16_to_f64(bits, lib=o.lib) == want, f"f16 0x{bits:04x}"
+    assert math.isinf(o.pkg.f16_to_f64(0x7C00, lib=o.lib))
+
+
+def pin_reconstruct_words(o):
+    r = _rng(1700)
+    atoms = r.normal(0, 1, (40, 6)).astype(np.float32)
+    idx = r.integers(0, 40, (5, 3, 4))
+    coeff = r.normal(0, 1, (5, 3, 4)).astype(np.float16)
+    coeff[0, 0, 3] = 0.0                                        # a padding word
+    idx[0, 0, 3] = 39
+    got = o.reconstruct(_pack(idx, coeff), atoms)
+    want = np.einsum("rgw,rgwd->rgd", coeff.astype(np.float64), atoms[idx].astype(np.float64))
+    _close(got, want, rtol=1e-14, atol=1e-14, what="reconstruct")
+    # one-hot codes with coefficient 1 give the atom back exactly
+    one = o.reconstruct(_pack(np.array([[7], [3]]), np.array([[1.0], [1.0]])), atoms)
+    assert np.array_equal(one, atoms[[7, 3]].astype(np.float64))
+
+
+def pin_coded_attention_is_plain_attention(o):
+    # atoms = the cache's own rows and one-hot codes: the coded path must equal
+    # plain attention over that cache
+    H, G, D = 4, 2, 5
+    q, k, v, off = _tiny(1800, [6, 9], H, G, D)
+    R = off[-1]
+    k_atoms = k.reshape(R * G, D)
+    v_atoms = v.reshape(R * G, D)
+    codes = _pack(np.arange(R * G).reshape(R, G, 1), np.ones((R, G, 1)))
+    st = o.pkg.coded_decode_attend(q, codes, codes, k_atoms, v_atoms, off, H, G, 0.8, lib=o.lib)
+    ref = o.attend(q, k, v, off, H, G, score_scale=0.8)
+    assert np.array_equal(st.out, ref.out), "coded one-hot = plain"
+
+
 ALL_PINS = [pin_bf16_widening, pin_brute_force_tiny, pin_single_key, pin_constant_v,
             pin_zero_query_mean, pin_two_key_closed_form, pin_group_symmetry, pin_merge_union,
             pin_carry_identity, pin_shift_invariance, pin_needle, pin_rows_subset,
             pin_bias_brute_force, pin_bias_constant_is_shift, pin_bias_mask_is_subset,
-            pin_topk_to_bias, pin_append_then_attend]
+            pin_topk_to_bias, pin_append_then_attend, pin_f16_coefficients, pin_reconstruct_words,
+            pin_coded_attention_is_plain_attention]
 
 
 def run_all(o):

@@ -17,7 +17,8 @@ from oracle import build as oracle_build
 MUTATIONS = {1: "interleaved head map", 2: "scale dropped", 3: "carry sign flipped",
              4: "not divided by partition", 5: "cache layout transposed",
              6: "merge without rescaling", 7: "last key dropped", 8: "keys used as values",
-             9: "bias inside the scale", 10: "top-k admits one past the end"}
+             9: "bias inside the scale", 10: "top-k admits one past the end",
+             11: "code word fields swapped"}
 
 
 @pytest.mark.parametrize("mutation", sorted(MUTATIONS), ids=lambda m: MUTATIONS[m])
