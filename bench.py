@@ -46,10 +46,13 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c2_bf16")
-    ap.add_argument("--op", choices=["attend", "append_attend", "masked_attend"], default="attend",
+    ap.add_argument("--op", choices=["attend", "append_attend", "masked_attend", "coded_attend"],
+                    default="attend",
                     help="attend: plain decode attention (the default line); append_attend: "
                          "append the new token's K/V then attend; masked_attend: index rows -> "
-                         "bias (gqa_topk_to_bias) then attend with it")
+                         "bias (gqa_topk_to_bias) then attend with it; coded_attend: the "
+                         "same shape as a dictionary-coded cache (8 code words per row, 256 "
+                         "atoms), KV bytes = code bytes read")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--e2e-steps", type=int, default=30)
@@ -252,6 +255,19 @@ def run_ours(args):
                         dtype=torch.int32).to(dev)
     bias = torch.zeros(w.total_rows, dtype=torch.float32, device=dev)
 
+    if args.op == "coded_attend":
+        # synthetic dictionary and codes of the workload's shape: 8 words per row
+        words, n_atoms = 8, 256
+        cg = torch.Generator().manual_seed(78)
+        idx = torch.randint(0, n_atoms, (w.total_rows, G, words), generator=cg, dtype=torch.int64)
+        cf = torch.randn((w.total_rows, G, words), generator=cg).to(torch.float16).view(torch.int16)
+        code = ((idx << 16) | (cf.to(torch.int64) & 0xFFFF)).to(torch.int64)
+        code = torch.where(code >= 2**31, code - 2**32, code).to(torch.int32)
+        kcodes = [code.to(dev).contiguous()]
+        vcodes = [torch.roll(code, 1, 0).to(dev).contiguous()]
+        atoms = torch.nn.functional.normalize(torch.randn((n_atoms, D), generator=cg), dim=1).to(dev)
+        kv_bytes = 2 * kcodes[0].numel() * 4
+
     def step(i):
         run_op(*caches[i % len(caches)])
 
@@ -262,7 +278,11 @@ def run_ours(args):
 
     def run_op(k, v, st=None):
         st = st or stream
-        if args.op == "append_attend":
+        if args.op == "coded_attend":
+            gqa.gqa_decode_attend_coded(q, kcodes[0], vcodes[0], atoms, atoms, offsets, H, G,
+                                        score_scale=w.score_scale, carry=carry, out=out,
+                                        max_seq_len=w.max_seq_len, workspace=ws, stream=st, flags=flags)
+        elif args.op == "append_attend":
             gqa.gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, H, G, score_scale=w.score_scale,
                                          carry=carry, out=out, max_seq_len=w.max_seq_len, workspace=ws,
                                          stream=st, flags=flags)

@@ -9,7 +9,8 @@ The entry points keep the C names:
   gqa_decode_attend, gqa_decode_append_attend, gqa_topk_to_bias,
   gqa_decode_workspace_size, gqa_workspace_init, gqa_softmax_merge,
   gqa_state_finalize, gqa_get_device_error, gqa_plan_splits,
-  gqa_status_string, gqa_version, gqa_decode_attend_static_workspace.
+  gqa_status_string, gqa_version, gqa_decode_attend_static_workspace,
+  gqa_softmax_merge_gathered, gqa_decode_attend_coded.
 
 If the compiled library is missing the first call raises ``LibraryMissing``;
 there is no fallback implementation.
@@ -21,7 +22,7 @@ import os
 __all__ = [
     "GqaError", "LibraryMissing", "State", "Workspace", "gqa_decode_attend",
     "gqa_decode_append_attend", "gqa_topk_to_bias", "gqa_decode_attend_static_workspace",
-    "gqa_softmax_merge_gathered",
+    "gqa_softmax_merge_gathered", "gqa_decode_attend_coded",
     "gqa_decode_workspace_size", "gqa_workspace_init", "gqa_softmax_merge", "gqa_state_finalize",
     "gqa_get_device_error", "gqa_plan_splits", "gqa_status_string", "gqa_version", "lib_path",
     "load_library",
@@ -37,6 +38,7 @@ GQA_ERR_DEVICE = 3
 GQA_ERR_WORKSPACE = 4
 GQA_ERR_BAD_OFFSETS = 5
 GQA_ERR_TIMEOUT = 6
+GQA_ERR_BAD_CODES = 7
 GQA_F32 = 0
 GQA_BF16 = 1
 GQA_FLAG_EARLY_START = 1
@@ -75,6 +77,11 @@ class _CParams(ctypes.Structure):
     ]
 
 
+class _CCodes(ctypes.Structure):
+    _fields_ = [("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p), ("words", ctypes.c_int32),
+                ("k_atoms", ctypes.c_void_p), ("v_atoms", ctypes.c_void_p), ("n_atoms", ctypes.c_int32)]
+
+
 _lib = None
 
 
@@ -100,6 +107,7 @@ def load_library(path=None):
     lib.gqa_workspace_init.argtypes = [sp, ctypes.c_size_t, sp]
     lib.gqa_decode_attend.argtypes = [ctypes.POINTER(_CParams), sp]
     lib.gqa_decode_append_attend.argtypes = [ctypes.POINTER(_CParams), sp, sp, sp]
+    lib.gqa_decode_attend_coded.argtypes = [ctypes.POINTER(_CParams), ctypes.POINTER(_CCodes), sp]
     lib.gqa_topk_to_bias.argtypes = [sp, i32, i32, sp, i32, sp, sp, sp]
     lib.gqa_softmax_merge.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
     lib.gqa_softmax_merge_gathered.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
@@ -111,7 +119,8 @@ def load_library(path=None):
     lib.gqa_version.argtypes = []
     for fn in ("gqa_decode_workspace_size", "gqa_workspace_init", "gqa_decode_attend", "gqa_softmax_merge",
                "gqa_state_finalize", "gqa_get_device_error", "gqa_plan_splits",
-               "gqa_decode_append_attend", "gqa_topk_to_bias", "gqa_softmax_merge_gathered"):
+               "gqa_decode_append_attend", "gqa_topk_to_bias", "gqa_softmax_merge_gathered",
+               "gqa_decode_attend_coded"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gqa_version.restype = ctypes.c_int32
     if path is None:
@@ -333,6 +342,44 @@ def gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_h
                         score_scale, carry, state_out, out, out_dtype, None, want_out, num_splits,
                         max_seq_len, max_len, workspace, stream, bias,
                         extra=(ctypes.c_void_p(_ptr(k_new)), ctypes.c_void_p(_ptr(v_new))), flags=flags)
+
+
+def gqa_decode_attend_coded(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_heads, num_kv_heads=0,
+                            *, score_scale=0.0, carry=None, state_out=None, out=None, out_dtype=None,
+                            partials_out=None, want_out=None, num_splits=0, max_seq_len=0,
+                            workspace=None, stream=None, bias=None, flags=0):
+    """Decode attention over a dictionary-coded cache: k_codes / v_codes int32
+    or uint32-as-int32 [max_len, G, words] (atom index << 16 | f16 coefficient
+    bits), k_atoms / v_atoms fp32 [n_atoms, D]; see include/gqa_decode.h."""
+    torch = _torch()
+    if want_out is None:
+        want_out = out is not None or (state_out is None and partials_out is None)
+    odt = _dtype_code(q) if out_dtype is None else _dtype_code(torch.empty(0, dtype=out_dtype))
+    if want_out and out is None:
+        out = torch.empty(q.shape, dtype=_torch_dtype(odt), device=q.device)
+    if out is not None:
+        odt = _dtype_code(out)
+    max_len = k_codes.shape[0]
+    p = _params(q, q, q, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
+                partials_out, num_splits, max_seq_len, max_len, bias, flags)
+    p.k = p.v = None
+    codes = _CCodes(_ptr(k_codes), _ptr(v_codes), k_codes.shape[-1], _ptr(k_atoms), _ptr(v_atoms),
+                    k_atoms.shape[0])
+    lib = load_library()
+    # workspace sizing sees the code arrays in the caches' place
+    pw = _params(q, q, q, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
+                 partials_out, num_splits, max_seq_len, max_len, bias, flags)
+    pw.k, pw.v = _ptr(k_codes), _ptr(v_codes)
+    nbytes = ctypes.c_size_t()
+    _check(lib.gqa_decode_workspace_size(ctypes.byref(pw), ctypes.byref(nbytes), None, None),
+           "gqa_decode_workspace_size")
+    ws = workspace or _default_workspace(q.device)
+    ws.reserve(nbytes.value, stream)
+    p.workspace = ws.ptr
+    p.workspace_bytes = ws.nbytes
+    _check(lib.gqa_decode_attend_coded(ctypes.byref(p), ctypes.byref(codes), _stream_handle(stream)),
+           "gqa_decode_attend_coded")
+    return out
 
 
 def gqa_topk_to_bias(idx, offsets, max_len, bias=None, workspace=None, stream=None):

@@ -61,6 +61,24 @@ cudaError_t prepare_f32(int* resident) {
                                                        C::kThreads, C::kSmemBytes);
 }
 
+constexpr int kCodedMaxSmem = 160 * 1024;     // qa + Wt tables: 2 * hpk * n_atoms floats
+
+template <int D, int HMAX>
+cudaError_t prepare_coded() {
+  return cudaFuncSetAttribute(gqa::gqa_partition_coded_kernel<D, HMAX>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kCodedMaxSmem);
+}
+
+cudaError_t prepare_coded_all() {
+  cudaError_t e = prepare_coded<64, 4>();
+  if (e == cudaSuccess) e = prepare_coded<64, 8>();
+  if (e == cudaSuccess) e = prepare_coded<64, 16>();
+  if (e == cudaSuccess) e = prepare_coded<128, 4>();
+  if (e == cudaSuccess) e = prepare_coded<128, 8>();
+  if (e == cudaSuccess) e = prepare_coded<128, 16>();
+  return e;
+}
+
 // Per-device one-time set-up (kernel attributes, occupancy, SM count).
 const DeviceInfo* device_info(int* dev_out) {
   int dev = -1;
@@ -79,6 +97,7 @@ const DeviceInfo* device_info(int* dev_out) {
   if (e == cudaSuccess) e = prepare_bf16<64, 2>(&di.resident_bf16[0][1]);
   if (e == cudaSuccess) e = prepare_bf16<128, 1>(&di.resident_bf16[1][0]);
   if (e == cudaSuccess) e = prepare_bf16<128, 2>(&di.resident_bf16[1][1]);
+  if (e == cudaSuccess) e = prepare_coded_all();
   if (e == cudaSuccess) e = prepare_f32<64, 16>(&di.resident_f32[0]);
   if (e == cudaSuccess) e = prepare_f32<128, 16>(&di.resident_f32[1]);
   if (e != cudaSuccess) {
@@ -481,6 +500,7 @@ const char* gqa_status_string(gqa_status s) {
     case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE";
     case GQA_ERR_BAD_OFFSETS: return "GQA_ERR_BAD_OFFSETS";
     case GQA_ERR_TIMEOUT: return "GQA_ERR_TIMEOUT";
+    case GQA_ERR_BAD_CODES: return "GQA_ERR_BAD_CODES";
   }
   return "GQA_ERR_UNKNOWN";
 }
@@ -537,6 +557,97 @@ gqa_status gqa_decode_append_attend(const gqa_decode_params* p, const void* k_ne
   if (!is_device_ptr(p->workspace)) return GQA_ERR_DEVICE;
   return attend_impl(p, r, static_cast<uint8_t*>(p->workspace), reinterpret_cast<cudaStream_t>(stream),
                      k_new, v_new);
+}
+
+gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_codes* codes,
+                                   gqa_stream_t stream) {
+  if (!p || !codes || p->struct_size != sizeof(gqa_decode_params)) return GQA_ERR_INVALID_ARGUMENT;
+  if (codes->words < 1 || codes->words > 64 || codes->n_atoms < 1 || codes->n_atoms > 65536)
+    return GQA_ERR_INVALID_ARGUMENT;
+  // Validate everything else as gqa_decode_attend would, with the code arrays
+  // standing in for the caches (their dtype is the queries').
+  gqa_decode_params pc = *p;
+  pc.k = codes->k_codes;
+  pc.v = codes->v_codes;
+  pc.kv_dtype = p->q_dtype;
+  Resolved r;
+  gqa_status st = resolve(&pc, &r, true);
+  if (st != GQA_OK) return st;
+  if (r.B > 0 && r.max_len > 0 && (!codes->k_atoms || !codes->v_atoms)) return GQA_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(codes->k_atoms) | reinterpret_cast<uintptr_t>(codes->v_atoms)) & 15u)
+    return GQA_ERR_SHAPE_MISMATCH;
+  const size_t smem = static_cast<size_t>(2) * r.hpk * codes->n_atoms * sizeof(float);
+  if (smem > static_cast<size_t>(kCodedMaxSmem)) return GQA_ERR_INVALID_ARGUMENT;   // hpk * n_atoms <= 20480
+  if (!p->workspace || p->workspace_bytes < r.bytes) return GQA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
+  const void* ptrs[] = {p->q, p->offsets, p->out, p->workspace, p->bias, codes->k_codes, codes->v_codes,
+                        codes->k_atoms, codes->v_atoms, p->carry_in.m, p->carry_in.l, p->carry_in.acc,
+                        p->state_out.m, p->state_out.l, p->state_out.acc, p->partials_out.m,
+                        p->partials_out.l, p->partials_out.acc};
+  for (const void* q : ptrs)
+    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
+  if (r.B == 0) return GQA_OK;
+  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  PartitionArgs a{};
+  a.q = p->q;
+  a.offsets = p->offsets;
+  a.B = r.B;
+  a.H = r.H;
+  a.G = r.G;
+  a.hpk = r.hpk;
+  a.max_len = r.max_len;
+  a.chunk_len = r.chunk;
+  a.num_splits = r.S;
+  a.scale_log2 = r.scale * gqa::kLog2e;
+  if (r.has_partials) {
+    a.part_m = p->partials_out.m;
+    a.part_l = p->partials_out.l;
+    a.part_acc = p->partials_out.acc;
+    a.write_empty = 1;
+  } else {
+    a.part_m = reinterpret_cast<float*>(ws + r.off_m);
+    a.part_l = reinterpret_cast<float*>(ws + r.off_l);
+    a.part_acc = reinterpret_cast<float*>(ws + r.off_acc);
+  }
+  a.err = reinterpret_cast<uint32_t*>(ws);
+  a.merge = r.want_merge ? 1 : 0;
+  a.counters = r.want_merge ? reinterpret_cast<uint32_t*>(ws + r.off_counters) : nullptr;
+  const bool has_carry = state_present(p->carry_in);
+  a.cm = has_carry ? p->carry_in.m : nullptr;
+  a.cl = has_carry ? p->carry_in.l : nullptr;
+  a.cacc = has_carry ? p->carry_in.acc : nullptr;
+  const bool has_so = state_present(p->state_out);
+  a.om = has_so ? p->state_out.m : nullptr;
+  a.ol = has_so ? p->state_out.l : nullptr;
+  a.oacc = has_so ? p->state_out.acc : nullptr;
+  a.out = p->out;
+  a.out_bf16 = r.out_bf16;
+  a.bias = p->bias;
+  gqa::CodedArgs c{codes->k_codes, codes->v_codes, codes->k_atoms, codes->v_atoms, codes->words,
+                   codes->n_atoms, r.bf16 ? 1 : 0};
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (r.clear_counters &&
+      cudaMemsetAsync(a.counters, 0, static_cast<size_t>(r.B) * r.G * sizeof(uint32_t), cs) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  const unsigned grid = static_cast<unsigned>(r.B) * r.S * r.G;
+  Launch l(grid, 256, smem, cs, (p->flags & GQA_FLAG_EARLY_START) != 0);
+  cudaError_t e;
+  const int hp = r.hpk <= 4 ? 4 : (r.hpk <= 8 ? 8 : 16);
+  if (r.D == 128)
+    e = hp == 4 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<128, 4>, a, c)
+      : hp == 8 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<128, 8>, a, c)
+                : cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<128, 16>, a, c);
+  else
+    e = hp == 4 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<64, 4>, a, c)
+      : hp == 8 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<64, 8>, a, c)
+                : cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<64, 16>, a, c);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  return GQA_OK;
 }
 
 gqa_status gqa_topk_to_bias(const int32_t* idx, int32_t batch, int32_t width, const int32_t* offsets,
@@ -637,6 +748,7 @@ gqa_status gqa_get_device_error(void* workspace, gqa_stream_t stream) {
   }
   if (word & gqa::kErrBadOffsets) return GQA_ERR_BAD_OFFSETS;
   if (word & gqa::kErrTimeout) return GQA_ERR_TIMEOUT;
+  if (word & gqa::kErrBadCodes) return GQA_ERR_BAD_CODES;
   return GQA_OK;
 }
 

@@ -64,7 +64,8 @@ typedef enum {
   GQA_ERR_DEVICE = 3,           /* pointer not device memory, no device, launch failure */
   GQA_ERR_WORKSPACE = 4,        /* workspace missing or smaller than required  */
   GQA_ERR_BAD_OFFSETS = 5,      /* device-detected: offsets not monotone / beyond max_len */
-  GQA_ERR_TIMEOUT = 6           /* device-detected: a pipeline wait gave up    */
+  GQA_ERR_TIMEOUT = 6,          /* device-detected: a pipeline wait gave up    */
+  GQA_ERR_BAD_CODES = 7         /* device-detected: a code word names a missing atom */
 } gqa_status;
 
 typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
@@ -206,6 +207,35 @@ gqa_status gqa_decode_attend_static_workspace(const gqa_decode_params* params, g
 gqa_status gqa_decode_append_attend(const gqa_decode_params* params, const void* k_new,
                                     const void* v_new, gqa_stream_t stream);
 
+/* A dictionary-coded KV cache (qualiaDB KvDictionary: a learned dictionary of
+ * atoms; `reconstruct_from_words` is the f16-coefficient inverse of
+ * `encode_to_words`, the compressed-cache read path). Every cache row of every
+ * KV head is `words` 32-bit code words; a word holds the atom index in its high
+ * 16 bits and the coefficient's IEEE binary16 bits in its low 16, and the row is
+ * sum_w coeff_w * atoms[index_w] (a zero coefficient, as in padding words,
+ * contributes nothing). K and V have their own dictionaries (pass the same
+ * pointer twice for one shared dictionary). All device memory. */
+typedef struct {
+  const uint32_t* k_codes;   /* [max_len, num_kv_heads, words] */
+  const uint32_t* v_codes;   /* [max_len, num_kv_heads, words] */
+  int32_t words;             /* code words per row, 1..64 */
+  const float* k_atoms;      /* [n_atoms, head_dim] fp32, 16-byte aligned */
+  const float* v_atoms;      /* [n_atoms, head_dim] fp32, 16-byte aligned */
+  int32_t n_atoms;           /* 1..65536, and heads_per_kv * n_atoms <= 20480 */
+} gqa_kv_codes;
+
+/* Decode attention over a dictionary-coded cache: exactly gqa_decode_attend on
+ * the reconstructed rows, computed from the codes without rebuilding them
+ * (logits from a table of each query head against every K atom; values as
+ * per-atom weights applied to the V atoms once). params->k, ->v and ->kv_dtype
+ * are ignored; q is fp32 or bf16; everything else (offsets, carry, bias,
+ * partials, outputs, workspace, flags) as gqa_decode_attend. A code word naming
+ * an atom >= n_atoms is skipped and flags GQA_ERR_BAD_CODES in the device error
+ * word. The per-atom sums use shared-memory atomics, so results are not
+ * bit-reproducible from run to run (they stay within the fp32 tolerance). */
+gqa_status gqa_decode_attend_coded(const gqa_decode_params* params, const gqa_kv_codes* codes,
+                                   gqa_stream_t stream);
+
 /* Index-selected attention as an additive bias (metrale glm5next_dsa_ref,
  * `topk_to_mask`: the attention reads a mask built from an index row; repeated
  * indices collapse, the INVALID sentinel -1 and out-of-range entries drop).
@@ -249,7 +279,8 @@ gqa_status gqa_state_finalize(const gqa_state* state, int32_t rows, int32_t head
                               int32_t out_dtype, gqa_stream_t stream);
 
 /* Synchronise `stream`, read and clear the workspace's device error word.
- * Returns GQA_OK, GQA_ERR_BAD_OFFSETS or GQA_ERR_TIMEOUT (the first set). */
+ * Returns GQA_OK, GQA_ERR_BAD_OFFSETS, GQA_ERR_TIMEOUT or GQA_ERR_BAD_CODES
+ * (the first set, in that order). */
 gqa_status gqa_get_device_error(void* workspace, gqa_stream_t stream);
 
 /* The split plan of the heuristic, exposed for inspection and tests (host only):
