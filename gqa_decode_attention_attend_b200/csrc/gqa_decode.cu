@@ -465,6 +465,16 @@ gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* w
   a.kw = const_cast<void*>(p->k);
   a.vw = const_cast<void*>(p->v);
   a.kv_elem = r.bf16 ? 2 : 4;
+  // A grid that fills most of the GPU's CTA slots lets the next kernel start
+  // when its last loads are issued (the next grid then only takes the few free
+  // slots and the stragglers' slots); a grid that leaves many slots free waits
+  // until its streams are done, or the next grid would split into an early and
+  // a late half (measured on B200: +2 % on 256 CTAs, -2..5 % on 160 CTAs).
+  {
+    const int64_t grid = static_cast<int64_t>(r.B) * r.S * r.G;
+    const int64_t slots = static_cast<int64_t>(r.sm_count) * r.per_sm;
+    a.trigger_at_last_load = (grid * 5 >= slots * 4) ? 1 : 0;
+  }
 
   // With no cache rows every tile is empty and no load is issued, but a tensor
   // map still needs a non-zero extent and a valid aligned base: the scratch

@@ -80,6 +80,10 @@ struct PartitionArgs {
   void* kw;
   void* vw;
   int32_t kv_elem;           // bytes per cache element (2 or 4)
+  // Where a CTA lets the next kernel on the stream be scheduled (early-start
+  // launches): 1 = once its producer has issued the tile's last load, 0 = once
+  // its consumers have finished the tile's cache stream.
+  int32_t trigger_at_last_load;
 };
 
 // Work item of a CTA: flattened index -> (b, split c, g), g fastest so that the
@@ -652,7 +656,7 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
       // next kernel on the stream may now be scheduled. It still waits for this
       // grid before reading what it writes, so its first cache loads overlap
       // this grid's last stages, epilogue and merges.
-      ptx::grid_launch_dependents();
+      if (a.trigger_at_last_load) ptx::grid_launch_dependents();
       if (*abort_flag) {
         // Drain the copies still in flight before the CTA's shared memory goes away.
         for (int it = max(0, issued - C::kStages); it < issued; ++it)
@@ -830,6 +834,9 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 
   // ------------------------------------------------------------ epilogue
+  // Otherwise the next kernel may be scheduled once the tile's cache stream is
+  // done, overlapping this grid's epilogue and merges.
+  if (!a.trigger_at_last_load && threadIdx.x == 0) ptx::grid_launch_dependents();
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
