@@ -409,20 +409,10 @@ cudaError_t launch_partition(const Resolved& r, const PartitionArgs& a, const CU
   return launch_f32<64, 16>(a, grid, st, early);
 }
 
-// Pointer checks and the single launch of a decode call, with the scratch at `ws`
-// (the caller's workspace, or the library's static array).
-gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* ws, cudaStream_t cs,
-                       const void* k_new = nullptr, const void* v_new = nullptr) {
-  const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out,
-                        p->carry_in.m, p->carry_in.l, p->carry_in.acc,
-                        p->state_out.m, p->state_out.l, p->state_out.acc,
-                        p->partials_out.m, p->partials_out.l, p->partials_out.acc,
-                        p->bias, k_new, v_new};
-  for (const void* q : ptrs)
-    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
-  if (r.B == 0) return GQA_OK;
-
-  PartitionArgs a;
+// Kernel arguments of a decode call whose scratch is at `ws`.
+PartitionArgs make_args(const gqa_decode_params* p, const Resolved& r, uint8_t* ws, const void* k_new,
+                        const void* v_new) {
+  PartitionArgs a{};
   a.q = p->q;
   a.k = p->k;
   a.v = p->v;
@@ -470,11 +460,26 @@ gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* w
   // slots and the stragglers' slots); a grid that leaves many slots free waits
   // until its streams are done, or the next grid would split into an early and
   // a late half (measured on B200: +2 % on 256 CTAs, -2..5 % on 160 CTAs).
-  {
-    const int64_t grid = static_cast<int64_t>(r.B) * r.S * r.G;
-    const int64_t slots = static_cast<int64_t>(r.sm_count) * r.per_sm;
-    a.trigger_at_last_load = (grid * 5 >= slots * 4) ? 1 : 0;
-  }
+  const int64_t grid = static_cast<int64_t>(r.B) * r.S * r.G;
+  const int64_t slots = static_cast<int64_t>(r.sm_count) * r.per_sm;
+  a.trigger_at_last_load = (grid * 5 >= slots * 4) ? 1 : 0;
+  return a;
+}
+
+// Pointer checks and the single launch of a decode call, with the scratch at `ws`
+// (the caller's workspace, or the library's static array).
+gqa_status attend_impl(const gqa_decode_params* p, const Resolved& r, uint8_t* ws, cudaStream_t cs,
+                       const void* k_new = nullptr, const void* v_new = nullptr) {
+  const void* ptrs[] = {p->q, p->k, p->v, p->offsets, p->out,
+                        p->carry_in.m, p->carry_in.l, p->carry_in.acc,
+                        p->state_out.m, p->state_out.l, p->state_out.acc,
+                        p->partials_out.m, p->partials_out.l, p->partials_out.acc,
+                        p->bias, k_new, v_new};
+  for (const void* q : ptrs)
+    if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
+  if (r.B == 0) return GQA_OK;
+
+  PartitionArgs a = make_args(p, r, ws, k_new, v_new);
 
   // With no cache rows every tile is empty and no load is issued, but a tensor
   // map still needs a non-zero extent and a valid aligned base: the scratch
@@ -598,41 +603,9 @@ gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_code
     if (!is_device_ptr(q)) return GQA_ERR_DEVICE;
   if (r.B == 0) return GQA_OK;
   uint8_t* ws = static_cast<uint8_t*>(p->workspace);
-  PartitionArgs a{};
-  a.q = p->q;
-  a.offsets = p->offsets;
-  a.B = r.B;
-  a.H = r.H;
-  a.G = r.G;
-  a.hpk = r.hpk;
-  a.max_len = r.max_len;
-  a.chunk_len = r.chunk;
-  a.num_splits = r.S;
-  a.scale_log2 = r.scale * gqa::kLog2e;
-  if (r.has_partials) {
-    a.part_m = p->partials_out.m;
-    a.part_l = p->partials_out.l;
-    a.part_acc = p->partials_out.acc;
-    a.write_empty = 1;
-  } else {
-    a.part_m = reinterpret_cast<float*>(ws + r.off_m);
-    a.part_l = reinterpret_cast<float*>(ws + r.off_l);
-    a.part_acc = reinterpret_cast<float*>(ws + r.off_acc);
-  }
-  a.err = reinterpret_cast<uint32_t*>(ws);
-  a.merge = r.want_merge ? 1 : 0;
-  a.counters = r.want_merge ? reinterpret_cast<uint32_t*>(ws + r.off_counters) : nullptr;
-  const bool has_carry = state_present(p->carry_in);
-  a.cm = has_carry ? p->carry_in.m : nullptr;
-  a.cl = has_carry ? p->carry_in.l : nullptr;
-  a.cacc = has_carry ? p->carry_in.acc : nullptr;
-  const bool has_so = state_present(p->state_out);
-  a.om = has_so ? p->state_out.m : nullptr;
-  a.ol = has_so ? p->state_out.l : nullptr;
-  a.oacc = has_so ? p->state_out.acc : nullptr;
-  a.out = p->out;
-  a.out_bf16 = r.out_bf16;
-  a.bias = p->bias;
+  PartitionArgs a = make_args(&pc, r, ws, nullptr, nullptr);
+  a.k = a.v = nullptr;
+  a.kw = a.vw = nullptr;
   gqa::CodedArgs c{codes->k_codes, codes->v_codes, codes->k_atoms, codes->v_atoms, codes->words,
                    codes->n_atoms, r.bf16 ? 1 : 0};
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
