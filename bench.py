@@ -84,13 +84,18 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# The sources that define the profiled launch of the bf16 partition kernel:
+# its body, the tile logic and fused merge it includes, the PTX wrappers, and
+# the host code that plans and launches it.
+PROFILED_SOURCES = ("gqa_decode.cu", "partition_bf16.cuh", "ptx.cuh", "tile.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gqa_decode_attention_attend_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in PROFILED_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -287,7 +292,7 @@ def run_ours(args):
                                          carry=carry, out=out, max_seq_len=w.max_seq_len, workspace=ws,
                                          stream=st, flags=flags)
         elif args.op == "masked_attend":
-            gqa.gqa_topk_to_bias(idx, offsets, w.total_rows, bias=bias, stream=st, flags=flags)
+            gqa.gqa_topk_to_bias(idx, offsets, w.total_rows, bias=bias, stream=st)
             gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
                                   out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st,
                                   bias=bias, flags=flags)

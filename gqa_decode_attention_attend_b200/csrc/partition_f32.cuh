@@ -65,11 +65,13 @@ gqa_partition_f32_kernel(const PartitionArgs a) {
       const float s2 = appended_logit2<D, float>(a, t, h, lane);
       if (lane == 0) smN[h] = s2;
     }
+    __syncthreads();   // smN is read by other warps in the epilogue (a warp may have no keys)
   }
-  // U keys per warp step: their loads are issued together, their per-head dot
-  // products reduced together (U-way interleaved butterflies), and the running
-  // state rescaled once per step.
-  constexpr int U = 4;
+  // U keys per warp step (32 floats of K and of V per lane: 16 keys at d 64,
+  // 8 at d 128): their loads are issued together, their per-head dot products
+  // reduced together (U-way interleaved butterflies), and the running state
+  // rescaled once per step.
+  constexpr int U = 32 / E;
 #pragma unroll 1
   for (int key0 = t.kbeg + warp; key0 < t.kstream; key0 += W * U) {
     float kv[U][E], vv[U][E];

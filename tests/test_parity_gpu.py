@@ -243,3 +243,18 @@ def test_final_output_dtype_bf16_from_fp32_inputs(dev):
     out, _ = gu.run(dw, out_dtype=torch.bfloat16)
     assert out.dtype == torch.bfloat16
     gu.check_out(out, ref, w, what="fp32 in, bf16 out")
+
+
+def test_stored_golden_values(dev):
+    """The fp32 workload against the oracle's stored values (tests/golden)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                    "c1_fp32_rows.json")))
+    w = workloads.config("c1_fp32")
+    dw = gu.DevWorkload(w, dev)
+    out, st = gu.run(dw, with_state=True)
+    ref = __import__("oracle").State(np.array(g["m"]), np.array(g["l"]), np.array(g["out"]) * np.array(g["l"])[:, None],
+                                     np.array(g["out"]))
+    gu.check_out(out, ref, w, what="golden c1")
+    gu.assert_close(st.m.cpu().numpy(), ref.m, torch.float32, "golden c1 m")
