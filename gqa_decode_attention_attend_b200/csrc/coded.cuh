@@ -28,15 +28,29 @@ struct CodedArgs {
   int32_t q_bf16;
 };
 
-// Word w of a code row: rows of a multiple of 4 words are read 16 bytes at a
-// time (the compiler merges the four reads of one quad), others word by word.
-__device__ __forceinline__ uint32_t code_word(const uint32_t* row, int w, int words) {
+constexpr int kMaxCodeWords = 16;
+
+// The words of one code row into registers (16-byte loads when the row is a
+// multiple of 4 words, else word by word); words past `words` are zero.
+__device__ __forceinline__ void load_code_row(const uint32_t* row, int words, uint32_t (&w)[kMaxCodeWords]) {
   if ((words & 3) == 0) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(row) + (w >> 2));
-    const int r = w & 3;
-    return r == 0 ? q.x : r == 1 ? q.y : r == 2 ? q.z : q.w;
+#pragma unroll
+    for (int q = 0; q < kMaxCodeWords / 4; ++q) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (4 * q < words) v = __ldg(reinterpret_cast<const uint4*>(row) + q);
+      w[4 * q] = v.x;
+      w[4 * q + 1] = v.y;
+      w[4 * q + 2] = v.z;
+      w[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kMaxCodeWords; ++i) w[i] = i < words ? __ldg(row + i) : 0u;
   }
-  return __ldg(row + w);
+}
+
+__device__ __forceinline__ float code_coeff(uint32_t word) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(word & 0xFFFFu)));
 }
 
 // Decode attention straight from the codes, never rebuilding a row:
@@ -45,16 +59,20 @@ __device__ __forceinline__ uint32_t code_word(const uint32_t* row, int w, int wo
 //   sum_j p_j V_j = sum_atom (sum_{j,w: i'_jw = atom} p_j c'_jw) vatom[atom]
 //     -- per-atom weights Wt[h][atom] accumulated per key (shared atomics),
 //     multiplied by the V atoms once at the end.
-// The online softmax runs per block of 256 keys (one key per thread): the
-// block's maximum per head, a rescale of l and Wt when it grows, then the
-// block's weights. Same tiles, partial states and fused merge as the other
-// partition kernels; the Wt sums are not bit-reproducible (atomic order).
-// Two CTAs per SM (registers capped at 128), as the split plan assumes.
+// The online softmax runs per block of 256 keys (one key per thread, its K and
+// V code rows fetched together): the block's maximum per head, a rescale of l
+// and Wt when it grows, then the block's weights. The atom tables are built
+// and applied by whole warps (lanes across D, one coalesced row per atom), so
+// both cost a few trips to L2 rather than one per atom. Same tiles, partial
+// states and fused merge as the other partition kernels; the Wt sums are not
+// bit-reproducible (atomic order). Two CTAs per SM (registers capped at 128),
+// as the split plan assumes.
 template <int D, int HMAX>
 __global__ void __launch_bounds__(256, 2) gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
-  constexpr int NT = 256, NW = NT / 32;
+  constexpr int NT = 256, NW = NT / 32, E = D / 32;
   extern __shared__ float csm[];
   __shared__ float qs[HMAX * D];
+  __shared__ float accb[HMAX * D];
   __shared__ float red[NW][HMAX];
   __shared__ float Mrun[HMAX], Lrun[HMAX], fac[HMAX];
   __shared__ float smM[16], smL[16], smC[16];
@@ -72,37 +90,42 @@ __global__ void __launch_bounds__(256, 2) gqa_partition_coded_kernel(const Parti
       merge_segment<D, HMAX>(a, t, 0, tid, smM, smL, smC, csm, hpk * NA, NamedSync128{});
     return;
   }
-  // query rows of the group, then the logit table against every K atom
+  // query rows of the group
   const size_t qrow = static_cast<size_t>(t.b) * a.H + static_cast<size_t>(t.g) * hpk;
-  for (int i = tid; i < hpk * D; i += NT)
+  for (int i = tid; i < hpk * D; i += NT) {
     qs[i] = c.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qrow * D + i])
                      : static_cast<const float*>(a.q)[qrow * D + i];
+    accb[i] = 0.f;
+  }
   if (tid < HMAX) {
     Mrun[tid] = -INFINITY;
     Lrun[tid] = 0.f;
   }
+  for (int i = tid; i < hpk * NA; i += NT) Wt[i] = 0.f;
   __syncthreads();
-  for (int at = tid; at < NA; at += NT) {
-    float dot[HMAX];
+  // the logit table: warp w takes atoms w, w+8, ...; lanes split D
+  {
+    float qreg[HMAX][E];
 #pragma unroll
-    for (int h = 0; h < HMAX; ++h) dot[h] = 0.f;
-    const float4* ka = reinterpret_cast<const float4*>(c.k_atoms + static_cast<size_t>(at) * D);
-#pragma unroll 4
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 kv = __ldg(ka + d4);
+    for (int h = 0; h < HMAX; ++h)
+#pragma unroll
+      for (int e = 0; e < E; ++e) qreg[h][e] = h < hpk ? qs[h * D + lane * E + e] : 0.f;
+#pragma unroll 2
+    for (int at = warp; at < NA; at += NW) {
+      float kv[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) kv[e] = __ldg(c.k_atoms + static_cast<size_t>(at) * D + lane * E + e);
 #pragma unroll
       for (int h = 0; h < HMAX; ++h) {
         if (h >= hpk) break;
-        const float* qh = qs + h * D + d4 * 4;
-        dot[h] = fmaf(qh[0], kv.x, fmaf(qh[1], kv.y, fmaf(qh[2], kv.z, fmaf(qh[3], kv.w, dot[h]))));
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) d = fmaf(qreg[h][e], kv[e], d);
+#pragma unroll
+        for (int x = 16; x >= 1; x >>= 1) d += __shfl_xor_sync(0xffffffffu, d, x);
+        if (lane == 0) qa[h * NA + at] = d * a.scale_log2;
       }
     }
-#pragma unroll
-    for (int h = 0; h < HMAX; ++h)
-      if (h < hpk) {
-        qa[h * NA + at] = dot[h] * a.scale_log2;
-        Wt[h * NA + at] = 0.f;
-      }
   }
   __syncthreads();
 
@@ -113,15 +136,19 @@ __global__ void __launch_bounds__(256, 2) gqa_partition_coded_kernel(const Parti
     const int key = kb + tid;
     const bool live = key < t.kend;
     const size_t crow = (static_cast<size_t>(t.o0) + (live ? key : t.kbeg)) * a.G + t.g;
+    uint32_t kw[kMaxCodeWords], vw[kMaxCodeWords];
+    if (live) {
+      load_code_row(c.k_codes + crow * W, W, kw);
+      load_code_row(c.v_codes + crow * W, W, vw);
+    }
     float sc[HMAX];
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) sc[h] = live ? 0.f : -INFINITY;
     if (live) {
-      const uint32_t* kc = c.k_codes + crow * W;
-      for (int w = 0; w < W; ++w) {
-        const uint32_t word = code_word(kc, w, W);
-        const int idx = static_cast<int>(word >> 16);
-        const float cf = __half2float(__ushort_as_half(static_cast<unsigned short>(word & 0xFFFFu)));
+#pragma unroll
+      for (int w = 0; w < kMaxCodeWords; ++w) {
+        const int idx = static_cast<int>(kw[w] >> 16);
+        const float cf = code_coeff(kw[w]);
         if (cf == 0.f) continue;
         if (idx >= NA) {
           bad = true;
@@ -180,11 +207,10 @@ __global__ void __launch_bounds__(256, 2) gqa_partition_coded_kernel(const Parti
       Lrun[tid] += ssum;
     }
     if (live) {
-      const uint32_t* vc = c.v_codes + crow * W;
-      for (int w = 0; w < W; ++w) {
-        const uint32_t word = code_word(vc, w, W);
-        const int idx = static_cast<int>(word >> 16);
-        const float cf = __half2float(__ushort_as_half(static_cast<unsigned short>(word & 0xFFFFu)));
+#pragma unroll
+      for (int w = 0; w < kMaxCodeWords; ++w) {
+        const int idx = static_cast<int>(vw[w] >> 16);
+        const float cf = code_coeff(vw[w]);
         if (cf == 0.f) continue;
         if (idx >= NA) {
           bad = true;
@@ -200,15 +226,39 @@ __global__ void __launch_bounds__(256, 2) gqa_partition_coded_kernel(const Parti
   if (bad) atomicOr(a.err, kErrBadCodes);
   if (threadIdx.x == 0) ptx::grid_launch_dependents();
 
-  // acc[h][d] = sum over atoms of Wt[h][atom] * vatom[atom][d]; the state goes
-  // out exactly as store_partial writes a single slot
+  // acc[h][d] = sum over atoms of Wt[h][atom] * vatom[atom][d]: warp w takes
+  // atoms w, w+8, ... with lanes across D, then the warps add into accb
+  {
+    float acc[HMAX][E];
+#pragma unroll
+    for (int h = 0; h < HMAX; ++h)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
+#pragma unroll 2
+    for (int at = warp; at < NA; at += NW) {
+      float vv[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) vv[e] = __ldg(c.v_atoms + static_cast<size_t>(at) * D + lane * E + e);
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h) {
+        if (h >= hpk) break;
+        const float wgt = Wt[h * NA + at];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[h][e] = fmaf(wgt, vv[e], acc[h][e]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < HMAX; ++h) {
+      if (h >= hpk) break;
+#pragma unroll
+      for (int e = 0; e < E; ++e) atomicAdd(accb + h * D + lane * E + e, acc[h][e]);
+    }
+  }
+  __syncthreads();
+  // the state goes out exactly as store_partial writes a single slot
   for (int i = tid; i < hpk * D; i += NT) {
     const int h = i / D, d = i % D;
-    const float* wr = Wt + h * NA;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int at = 0; at < NA; ++at) acc = fmaf(wr[at], __ldg(c.v_atoms + static_cast<size_t>(at) * D + d), acc);
-    a.part_acc[state_index(a, t, h) * D + d] = acc;
+    a.part_acc[state_index(a, t, h) * D + d] = accb[i];
   }
   if (tid < hpk) {
     const size_t si = state_index(a, t, tid);

@@ -577,7 +577,7 @@ gqa_status gqa_decode_append_attend(const gqa_decode_params* p, const void* k_ne
 gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_codes* codes,
                                    gqa_stream_t stream) {
   if (!p || !codes || p->struct_size != sizeof(gqa_decode_params)) return GQA_ERR_INVALID_ARGUMENT;
-  if (codes->words < 1 || codes->words > 64 || codes->n_atoms < 1 || codes->n_atoms > 65536)
+  if (codes->words < 1 || codes->words > 16 || codes->n_atoms < 1 || codes->n_atoms > 65536)
     return GQA_ERR_INVALID_ARGUMENT;
   // Validate everything else as gqa_decode_attend would, with the code arrays
   // standing in for the caches (their dtype is the queries').

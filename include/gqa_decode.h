@@ -218,7 +218,7 @@ gqa_status gqa_decode_append_attend(const gqa_decode_params* params, const void*
 typedef struct {
   const uint32_t* k_codes;   /* [max_len, num_kv_heads, words] */
   const uint32_t* v_codes;   /* [max_len, num_kv_heads, words] */
-  int32_t words;             /* code words per row, 1..64 */
+  int32_t words;             /* code words per row, 1..16 */
   const float* k_atoms;      /* [n_atoms, head_dim] fp32, 16-byte aligned */
   const float* v_atoms;      /* [n_atoms, head_dim] fp32, 16-byte aligned */
   int32_t n_atoms;           /* 1..65536, and heads_per_kv * n_atoms <= 20480 */

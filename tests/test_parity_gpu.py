@@ -258,3 +258,42 @@ def test_stored_golden_values(dev):
                                      np.array(g["out"]))
     gu.check_out(out, ref, w, what="golden c1")
     gu.assert_close(st.m.cpu().numpy(), ref.m, torch.float32, "golden c1 m")
+
+
+def test_more_segments_than_the_fixed_ticket_region(dev):
+    """9000 sequences x 8 KV heads = 72000 (sequence, KV head) segments: the merge
+    tickets then live in a region cleared on every call."""
+    g = torch.Generator().manual_seed(31)
+    lengths = torch.randint(1, 9, (9000,), generator=g).tolist()
+    lengths[5] = 300                       # one sequence long enough to split
+    w = workloads.make("many", lengths, 8, 8, 64, seed=32, carry=True)
+    dw = gu.DevWorkload(w, dev)
+    rows = list(range(0, 9000 * 8, 97)) + list(range(40, 48))
+    ref = gu.oracle_state(w, rows=rows)
+    for _ in range(2):                     # the second call must see cleared tickets again
+        out, st = gu.run(dw, with_state=True, out_dtype=torch.float32)
+        gu.check_out(out, ref, w, rows=rows, what="72000 segments")
+        gu.check_state(st, ref, w, rows=rows, what="72000 segments state")
+
+
+def test_partials_and_merged_output_together(dev):
+    w = workloads.make("both", [3000, 17, 1], 16, 4, 128, seed=33, carry=True)
+    dw = gu.DevWorkload(w, dev)
+    rows = w.batch * w.num_heads
+    parts = gqa.State.empty(rows, 128, dev, (5,))
+    out = gqa.gqa_decode_attend(dw.q, dw.k, dw.v, dw.offsets, 16, 4, carry=dw.carry, partials_out=parts,
+                                num_splits=5, max_seq_len=3000, out_dtype=torch.float32, want_out=True)
+    ref = gu.oracle_state(w)
+    gu.check_out(out, ref, w, what="out beside partials")
+    # the partials alone (no carry) merge to the carry-free result
+    merged = gqa.gqa_softmax_merge(parts)
+    gu.assert_close(merged.cpu().numpy(), gu.oracle_state(w, carry=False).out, torch.bfloat16,
+                    "partials beside out")
+
+
+def test_zero_kv_heads_means_one_per_query_head(dev):
+    w = workloads.make("mha", [500, 64], 8, 8, 64, seed=34)
+    dw = gu.DevWorkload(w, dev)
+    a = gqa.gqa_decode_attend(dw.q, dw.k, dw.v, dw.offsets, 8, 0, out_dtype=torch.float32)
+    b = gqa.gqa_decode_attend(dw.q, dw.k, dw.v, dw.offsets, 8, 8, out_dtype=torch.float32)
+    assert torch.equal(a, b)
