@@ -388,20 +388,24 @@ def run_ours(args):
 
     # ---- end to end: pinned host inputs -> device, call, output -> pinned host
     hq = w.q.pin_memory()
-    hk = w.k.pin_memory()
-    hv = w.v.pin_memory()
     hoff = w.offsets.pin_memory()
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dk, dv = caches[0]
-    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() * 2 + hoff.numel() * 4
+    # the step's cache inputs: the raw K/V, or the code arrays for the coded op
+    if args.op == "coded_attend":
+        dev_cache = [kcodes[0], vcodes[0]]
+    else:
+        dev_cache = list(caches[0])
+    host_cache = [t.cpu().pin_memory() for t in dev_cache]
+    h2d = (hq.numel() * hq.element_size() + sum(t.numel() * t.element_size() for t in host_cache) +
+           hoff.numel() * 4)
     d2h = hout.numel() * hout.element_size()
 
     def e2e_step():
         q.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
+        for d, h in zip(dev_cache, host_cache):
+            d.copy_(h, non_blocking=True)
         offsets.copy_(hoff, non_blocking=True)
-        run_op(dk, dv)
+        run_op(*caches[0])
         hout.copy_(out, non_blocking=True)
 
     n_e2e = 0 if args.quick else args.e2e_steps

@@ -201,8 +201,12 @@ def _c_state(s):
 
 class Workspace:
     """Scratch memory for gqa_decode_attend: a uint8 device tensor, 256-byte
-    aligned, whose error word is zeroed once by gqa_workspace_init. It grows on
-    demand (and is then re-initialised)."""
+    aligned, zeroed once by gqa_workspace_init (error word and merge tickets).
+    It grows on demand (and is then re-initialised); growing frees the old
+    buffer in the current stream's order, so a workspace belongs to one stream.
+    Calls that may run at the same time (other streams, other threads) need
+    workspaces of their own: the functions below fall back to one default
+    workspace per device when none is given."""
 
     def __init__(self, device, nbytes=256):
         self.device = device
