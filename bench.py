@@ -9,13 +9,19 @@ N(0,1), bf16 output. Inputs are resident in HBM before the timed region; two
 copies of the 256 MiB cache are alternated so consecutive steps never read a
 cache the 126 MB L2 could still hold.
 
+The K timed steps are captured once into a CUDA graph and replayed (the call
+allocates nothing and never synchronises), each launched with
+GQA_FLAG_EARLY_START (no step writes the cache rows or offsets the next one
+reads); --eager and --no-early-start turn either off.
+
 Prints ONE JSON line (rank 0). `value` is the KV-cache bytes read per step,
 summed over ranks, divided by the max-over-ranks device time (GB/s); `e2e` is
 the same metric through the same public call when every step also copies its
 inputs from pinned host memory and its output back.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--no-cpu-baseline]
+                  [--workload NAME] [--op OP] [--eager] [--no-early-start]
+                  [--no-cpu-baseline] [--quick]
 
 --impl reference times the f64 CPU oracle (the library's reference
 implementation) on a bounded sample of the same workload, on rank 0 only.

@@ -306,14 +306,21 @@ def _attend_call(entry, q, k, v, offsets, num_heads, num_kv_heads, score_scale, 
     p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
                 partials_out, num_splits, max_seq_len, max_len, bias, flags)
     lib = load_library()
-    nbytes = ctypes.c_size_t()
-    _check(lib.gqa_decode_workspace_size(ctypes.byref(p), ctypes.byref(nbytes), None, None),
-           "gqa_decode_workspace_size")
     ws = workspace or _default_workspace(q.device)
-    ws.reserve(nbytes.value, stream)
+    sh = _stream_handle(stream)
     p.workspace = ws.ptr
     p.workspace_bytes = ws.nbytes
-    _check(getattr(lib, entry)(ctypes.byref(p), *extra, _stream_handle(stream)), entry)
+    st = getattr(lib, entry)(ctypes.byref(p), *extra, sh)
+    if st == GQA_ERR_WORKSPACE:
+        # too small (checked before anything is launched): size it, grow, retry
+        nbytes = ctypes.c_size_t()
+        _check(lib.gqa_decode_workspace_size(ctypes.byref(p), ctypes.byref(nbytes), None, None),
+               "gqa_decode_workspace_size")
+        ws.reserve(nbytes.value, stream)
+        p.workspace = ws.ptr
+        p.workspace_bytes = ws.nbytes
+        st = getattr(lib, entry)(ctypes.byref(p), *extra, sh)
+    _check(st, entry)
     return out
 
 

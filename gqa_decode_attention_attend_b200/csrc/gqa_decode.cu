@@ -133,8 +133,22 @@ EncodeTiledFn encode_tiled() {
 }
 
 // K or V cache [max_len, G, D] bf16 as a 2-D tensor (G*D columns, max_len rows);
-// box = 64 columns (128 bytes, one swizzle span) x 64 rows.
+// box = 64 columns (128 bytes, one swizzle span) x 64 rows. The last few
+// encodings are kept per thread and reused for an identical cache.
 bool make_kv_map(CUtensorMap* m, const void* base, int max_len, int G, int D) {
+  struct Entry {
+    const void* base;
+    int max_len, G, D;
+    CUtensorMap map;
+  };
+  constexpr int kKept = 4;
+  thread_local Entry kept[kKept] = {};
+  thread_local int next = 0;
+  for (int i = 0; i < kKept; ++i)
+    if (kept[i].base == base && kept[i].max_len == max_len && kept[i].G == G && kept[i].D == D) {
+      *m = kept[i].map;
+      return true;
+    }
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(G) * D, static_cast<cuuint64_t>(max_len)};
@@ -144,19 +158,40 @@ bool make_kv_map(CUtensorMap* m, const void* base, int max_len, int G, int D) {
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  kept[next] = Entry{base, max_len, G, D, *m};
+  next = (next + 1) % kKept;
+  return true;
 }
 
 // ------------------------------------------------------------------ validation helpers
 
+// Whether `p` is device (or managed) memory. Addresses already seen to be
+// device memory are remembered in a small per-thread ring (64 entries), so a
+// decode loop that passes the same buffers call after call pays for the
+// driver query once; host addresses are never remembered.
 bool is_device_ptr(const void* p) {
   if (p == nullptr) return true;
+  constexpr int kSeen = 64;
+  thread_local const void* seen[kSeen] = {};
+  thread_local int seen_dev[kSeen] = {};
+  thread_local int next = 0;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  for (int i = 0; i < kSeen; ++i)
+    if (seen[i] == p && seen_dev[i] == dev) return true;
   cudaPointerAttributes at;
   if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
-  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+  const bool ok = at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+  if (ok) {
+    seen[next] = p;
+    seen_dev[next] = dev;
+    next = (next + 1) % kSeen;
+  }
+  return ok;
 }
 
 bool state_present(const gqa_state& s) { return s.m || s.l || s.acc; }
