@@ -61,21 +61,31 @@ cudaError_t prepare_f32(int* resident) {
                                                        C::kThreads, C::kSmemBytes);
 }
 
-constexpr int kCodedMaxSmem = 160 * 1024;     // qa + Wt tables: 2 * hpk * n_atoms floats
+// the coded kernel's largest dynamic shared memory: 16 code words, the largest tables
+constexpr int kCodedMaxSmem = static_cast<int>(gqa::coded_smem_bytes(gqa::kMaxCodeWords, 1,
+                                                                      gqa::kCodedMaxTableEntries));
 
-template <int D, int HMAX>
+template <int D, int HMAX, int MW>
 cudaError_t prepare_coded() {
-  return cudaFuncSetAttribute(gqa::gqa_partition_coded_kernel<D, HMAX>,
+  return cudaFuncSetAttribute(gqa::gqa_partition_coded_kernel<D, HMAX, MW>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, kCodedMaxSmem);
 }
 
+template <int D, int HMAX>
+cudaError_t prepare_coded_words() {
+  cudaError_t e = prepare_coded<D, HMAX, 4>();
+  if (e == cudaSuccess) e = prepare_coded<D, HMAX, 8>();
+  if (e == cudaSuccess) e = prepare_coded<D, HMAX, 16>();
+  return e;
+}
+
 cudaError_t prepare_coded_all() {
-  cudaError_t e = prepare_coded<64, 4>();
-  if (e == cudaSuccess) e = prepare_coded<64, 8>();
-  if (e == cudaSuccess) e = prepare_coded<64, 16>();
-  if (e == cudaSuccess) e = prepare_coded<128, 4>();
-  if (e == cudaSuccess) e = prepare_coded<128, 8>();
-  if (e == cudaSuccess) e = prepare_coded<128, 16>();
+  cudaError_t e = prepare_coded_words<64, 4>();
+  if (e == cudaSuccess) e = prepare_coded_words<64, 8>();
+  if (e == cudaSuccess) e = prepare_coded_words<64, 16>();
+  if (e == cudaSuccess) e = prepare_coded_words<128, 4>();
+  if (e == cudaSuccess) e = prepare_coded_words<128, 8>();
+  if (e == cudaSuccess) e = prepare_coded_words<128, 16>();
   return e;
 }
 
@@ -424,6 +434,21 @@ cudaError_t launch_f32(const PartitionArgs& a, unsigned grid, cudaStream_t st, b
   return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_f32_kernel<D, HMAX>, a);
 }
 
+// The coded kernel for heads_per_kv bound hp (4, 8, 16) and words bound mw (4, 8, 16).
+template <int D, int HMAX>
+cudaError_t launch_coded_hp(Launch& l, int mw, const PartitionArgs& a, const gqa::CodedArgs& c) {
+  if (mw == 4) return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 4>, a, c);
+  if (mw == 8) return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 8>, a, c);
+  return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 16>, a, c);
+}
+
+template <int D>
+cudaError_t launch_coded(Launch& l, int hp, int mw, const PartitionArgs& a, const gqa::CodedArgs& c) {
+  if (hp == 4) return launch_coded_hp<D, 4>(l, mw, a, c);
+  if (hp == 8) return launch_coded_hp<D, 8>(l, mw, a, c);
+  return launch_coded_hp<D, 16>(l, mw, a, c);
+}
+
 cudaError_t launch_partition(const Resolved& r, const PartitionArgs& a, const CUtensorMap* tk,
                              const CUtensorMap* tv, cudaStream_t st, bool early) {
   const unsigned grid = static_cast<unsigned>(r.B) * r.S * r.G;
@@ -626,8 +651,8 @@ gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_code
   if (r.B > 0 && r.max_len > 0 && (!codes->k_atoms || !codes->v_atoms)) return GQA_ERR_INVALID_ARGUMENT;
   if ((reinterpret_cast<uintptr_t>(codes->k_atoms) | reinterpret_cast<uintptr_t>(codes->v_atoms)) & 15u)
     return GQA_ERR_SHAPE_MISMATCH;
-  const size_t smem = static_cast<size_t>(2) * r.hpk * codes->n_atoms * sizeof(float);
-  if (smem > static_cast<size_t>(kCodedMaxSmem)) return GQA_ERR_INVALID_ARGUMENT;   // hpk * n_atoms <= 20480
+  if (static_cast<int64_t>(r.hpk) * codes->n_atoms > gqa::kCodedMaxTableEntries) return GQA_ERR_INVALID_ARGUMENT;
+  const size_t smem = gqa::coded_smem_bytes(codes->words, r.hpk, codes->n_atoms);
   if (!p->workspace || p->workspace_bytes < r.bytes) return GQA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
   const void* ptrs[] = {p->q, p->offsets, p->out, p->workspace, p->bias, codes->k_codes, codes->v_codes,
@@ -653,14 +678,8 @@ gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_code
   Launch l(grid, 256, smem, cs, (p->flags & GQA_FLAG_EARLY_START) != 0);
   cudaError_t e;
   const int hp = r.hpk <= 4 ? 4 : (r.hpk <= 8 ? 8 : 16);
-  if (r.D == 128)
-    e = hp == 4 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<128, 4>, a, c)
-      : hp == 8 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<128, 8>, a, c)
-                : cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<128, 16>, a, c);
-  else
-    e = hp == 4 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<64, 4>, a, c)
-      : hp == 8 ? cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<64, 8>, a, c)
-                : cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<64, 16>, a, c);
+  const int mw = codes->words <= 4 ? 4 : (codes->words <= 8 ? 8 : 16);
+  e = r.D == 128 ? launch_coded<128>(l, hp, mw, a, c) : launch_coded<64>(l, hp, mw, a, c);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_DEVICE;

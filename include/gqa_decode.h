@@ -221,7 +221,7 @@ typedef struct {
   int32_t words;             /* code words per row, 1..16 */
   const float* k_atoms;      /* [n_atoms, head_dim] fp32, 16-byte aligned */
   const float* v_atoms;      /* [n_atoms, head_dim] fp32, 16-byte aligned */
-  int32_t n_atoms;           /* 1..65536, and heads_per_kv * n_atoms <= 20480 */
+  int32_t n_atoms;           /* 1..65536, and heads_per_kv * n_atoms <= 12288 */
 } gqa_kv_codes;
 
 /* Decode attention over a dictionary-coded cache: exactly gqa_decode_attend on
@@ -231,8 +231,9 @@ typedef struct {
  * are ignored; q is fp32 or bf16; everything else (offsets, carry, bias,
  * partials, outputs, workspace, flags) as gqa_decode_attend. A code word naming
  * an atom >= n_atoms is skipped and flags GQA_ERR_BAD_CODES in the device error
- * word. The per-atom sums use shared-memory atomics, so results are not
- * bit-reproducible from run to run (they stay within the fp32 tolerance). */
+ * word. The per-atom value weights are summed per block of 256 keys in 32-bit
+ * fixed point, scaled to the block's largest possible sum (rounding error at
+ * most 2^-31 of it per weight), so results are bit-reproducible. */
 gqa_status gqa_decode_attend_coded(const gqa_decode_params* params, const gqa_kv_codes* codes,
                                    gqa_stream_t stream);
 

@@ -78,3 +78,45 @@ def test_bad_code_is_flagged():
     ws = gqa.Workspace(dev, 1 << 20)
     run_coded(w, kc, vc, ka, va, dev, workspace=ws)
     assert gqa.gqa_get_device_error(ws) == gqa.GQA_ERR_BAD_CODES
+
+
+def test_coded_is_deterministic():
+    """The value weights are summed in fixed point by integer atomics, whose
+    sums do not depend on their order: repeated calls give identical bits."""
+    dev = gu.device()
+    w = workloads.make("cdet", [4096] * 4, 32, 8, 128, seed=8, carry=True)
+    kc, vc, ka, va = make_codes(w.total_rows, 8, 8, 256, 128, seed=9)
+    outs = [run_coded(w, kc, vc, ka, va, dev, out_dtype=torch.float32) for _ in range(4)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
+@pytest.mark.parametrize("words", [6, 3])
+def test_coded_sharp_softmax_and_wide_coefficients(words):
+    """Peaked logits (score scale 1 instead of 1/sqrt(128): few keys carry the
+    weight) and coefficients spread over four and a half orders of magnitude,
+    at the fp32 tolerance: the fixed-point scale of each block follows the
+    weights actually present."""
+    dev = gu.device()
+    D, H, G, NA = 128, 16, 4, 96
+    lengths = [1500, 257, 2100]
+    w = workloads.make("csharp", lengths, H, G, D, dtype=torch.float32, seed=10 + words,
+                       score_scale=1.0, carry=True)
+    rng = np.random.default_rng(11 + words)
+    ka = rng.normal(0, 1, (NA, D))
+    va = rng.normal(0, 1, (NA, D))
+    ka = (ka / np.linalg.norm(ka, axis=1, keepdims=True)).astype(np.float32)
+    va = (va / np.linalg.norm(va, axis=1, keepdims=True)).astype(np.float32)
+
+    def codes():
+        idx = rng.integers(0, NA, (w.total_rows, G, words)).astype(np.uint32)
+        mag = 10.0 ** rng.uniform(-4, 0.5, (w.total_rows, G, words))
+        cf = (mag * rng.choice([-1.0, 1.0], mag.shape)).astype(np.float16)
+        return (idx << 16) | cf.view(np.uint16).astype(np.uint32)
+
+    kc, vc = codes(), codes()
+    ref = oracle.coded_decode_attend(workloads.host_array(w.q), kc, vc, ka, va, w.offsets.numpy(), H, G,
+                                     score_scale=1.0, carry=tuple(t.numpy() for t in w.carry))
+    out = run_coded(w, kc, vc, ka, va, dev, out_dtype=torch.float32, score_scale=1.0)
+    gu.assert_close(out.reshape(-1, D).cpu().numpy(), ref.out, torch.float32, f"sharp coded words{words}")
