@@ -460,10 +460,12 @@ def run_ours(args):
             "pct_of_nominal_8tbs": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
             "pct_of_measured_peak": round(100.0 * value / world / peak, 2),
             "roofline": {
-                "bound": "hbm", "kernel": "gqa_partition_bf16_kernel" if w.k.dtype == torch.bfloat16
-                else "gqa_partition_f32_kernel",
+                "bound": "hbm",
+                "kernel": ("gqa_partition_coded_kernel" if args.op == "coded_attend" else
+                           "gqa_partition_bf16_kernel" if w.k.dtype == torch.bfloat16
+                           else "gqa_partition_f32_kernel"),
                 "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_src, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name) if args.op == "attend" else None,
                 "algorithmic_bytes_per_launch": kv_bytes, "launch_ms": launch_ms,
                 "partials_only_launch_ms": part_ms,
                 "partials_only_gbs": round(kv_bytes / (part_ms / 1e3) / 1e9, 1),
