@@ -19,8 +19,9 @@
 //  * gqa_merge_kernel<D>: the standalone merge of caller-held states and a
 //    carry (USearch linear algebra, DenseAttendConfig::carry: partial-softmax
 //    rescaling), optional state out, optional out = acc / l.
-//  * gqa_partition_coded_kernel<D, HMAX>: the same tiles over a
-//    dictionary-coded cache (qualiaDB KvDictionary read path).
+//  * gqa_partition_coded_kernel<D, HMAX, MW>: the same tiles over a
+//    dictionary-coded cache (qualiaDB KvDictionary read path): logits by table
+//    lookup, value weights summed in fixed point with 32-bit shared atomics.
 //  * gqa_topk_to_bias_kernel: index rows -> additive bias (metrale
 //    glm5next_dsa_ref, topk_to_mask).
 //
