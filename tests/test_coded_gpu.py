@@ -120,3 +120,20 @@ def test_coded_sharp_softmax_and_wide_coefficients(words):
                                      score_scale=1.0, carry=tuple(t.numpy() for t in w.carry))
     out = run_coded(w, kc, vc, ka, va, dev, out_dtype=torch.float32, score_scale=1.0)
     gu.assert_close(out.reshape(-1, D).cpu().numpy(), ref.out, torch.float32, f"sharp coded words{words}")
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_coded_at_the_table_limit(D):
+    """heads_per_kv * n_atoms = 12288 with 16 words per row: the largest
+    shared-memory footprint the kernel accepts; one atom more is refused."""
+    dev = gu.device()
+    H, G, NA, words = 16, 1, 768, 16
+    w = workloads.make("climit", [300, 17, 0], H, G, D, dtype=torch.float32, seed=12, carry=True)
+    kc, vc, ka, va = make_codes(w.total_rows, G, words, NA, D, seed=13)
+    ref = oracle.coded_decode_attend(workloads.host_array(w.q), kc, vc, ka, va, w.offsets.numpy(), H, G,
+                                     carry=tuple(t.numpy() for t in w.carry))
+    out = run_coded(w, kc, vc, ka, va, dev, out_dtype=torch.float32)
+    gu.assert_close(out.reshape(-1, D).cpu().numpy(), ref.out, torch.float32, f"coded at the limit D{D}")
+    ka2 = np.concatenate([ka, ka[:1]])
+    with pytest.raises(gqa.GqaError):
+        run_coded(w, kc, vc, ka2, ka2, dev, out_dtype=torch.float32)
