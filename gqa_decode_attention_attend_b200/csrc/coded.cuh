@@ -80,9 +80,10 @@ __device__ __forceinline__ float block_weight_scale(float bound) {
 // depend on their order; barrier); at the next block's start Wb is folded
 // into the float table Wt, rescaled to the new running maximum. The partition
 // l is kept per thread and reduced once. So the coded kernel's results are
-// bit-reproducible. The logit table is built one atom per thread (q read from
-// shared memory, no cross-lane sums); the V atoms are applied by whole warps
-// (lanes across D, eight atoms in flight). Same tiles, partial states and
+// bit-reproducible. The logit table is built by whole warps, lanes across D
+// (coalesced atom rows), with a warp reduce-scatter of the partial dot
+// products; the V atoms are applied by whole warps the same way (lanes across
+// D, no cross-lane sums). Same tiles, partial states and
 // fused merge as the other partition kernels. Two CTAs per SM for the usual
 // table sizes (registers capped at 128), as the split plan assumes.
 // MW: a compile-time bound on the words per row (4, 8 or 16) for the per-key loops.
@@ -172,29 +173,50 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
     Wb[i] = 0u;
   }
   __syncthreads();
-  // the logit table, one atom per thread: its row streamed in float4 steps
-  // (eight in flight), q broadcast from shared memory
-  for (int at = tid; at < NA; at += NT) {
-    const float4* kr = reinterpret_cast<const float4*>(c.k_atoms + static_cast<size_t>(at) * D);
-    float d[HMAX];
-#pragma unroll
-    for (int h = 0; h < HMAX; ++h) d[h] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < D / 4; ++j) {
-      const float4 kv = __ldg(kr + j);
-#pragma unroll
-      for (int h = 0; h < HMAX; ++h) {
-        if (h >= hpk) break;
-        const float4 qv = *reinterpret_cast<const float4*>(qs + h * D + 4 * j);
-        d[h] = fmaf(qv.x, kv.x, d[h]);
-        d[h] = fmaf(qv.y, kv.y, d[h]);
-        d[h] = fmaf(qv.z, kv.z, d[h]);
-        d[h] = fmaf(qv.w, kv.w, d[h]);
-      }
-    }
+  // the logit table: a warp takes A = 32 / HMAX atoms per pass, lanes across D
+  // (coalesced rows, two passes of loads in flight). Each lane's A x HMAX
+  // partial dot products are summed across the warp by a reduce-scatter: at
+  // each of 5 steps a lane keeps half of its values and adds the other half
+  // from the lane `off` away, so lane L ends with atom L / HMAX, head L % HMAX.
+  {
+    constexpr int A = 32 / HMAX;
+    float qreg[HMAX][E];
 #pragma unroll
     for (int h = 0; h < HMAX; ++h)
-      if (h < hpk) qa[h * NA + at] = d[h] * a.scale_log2;
+#pragma unroll
+      for (int e = 0; e < E; ++e) qreg[h][e] = h < hpk ? qs[h * D + lane * E + e] : 0.f;
+#pragma unroll 2
+    for (int a0 = warp * A; a0 < NA; a0 += NW * A) {
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < A; ++i) {
+        float kv[E];
+        const int at = a0 + i;
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          kv[e] = at < NA ? __ldg(c.k_atoms + static_cast<size_t>(at) * D + lane * E + e) : 0.f;
+#pragma unroll
+        for (int h = 0; h < HMAX; ++h) {
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) d = fmaf(qreg[h][e], kv[e], d);
+          v[i * HMAX + h] = d;
+        }
+      }
+#pragma unroll
+      for (int st = 0; st < 5; ++st) {
+        const int off = 16 >> st;
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+          const float send = upper ? v[i] : v[i + off];
+          const float keep = upper ? v[i + off] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      const int at = a0 + lane / HMAX, h = lane % HMAX;
+      if (at < NA && h < hpk) qa[h * NA + at] = v[0] * a.scale_log2;
+    }
   }
   __syncthreads();
 
@@ -359,7 +381,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
     for (int h = 0; h < HMAX; ++h)
 #pragma unroll
       for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
-#pragma unroll 8
+#pragma unroll 16
     for (int at = warp; at < NA; at += NW) {
       float vv[E];
 #pragma unroll
