@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c2_bf16")
+    ap.add_argument("--workload", default="bf16_b16_n4096")
     ap.add_argument("--op", choices=["attend", "append_attend", "masked_attend", "coded_attend"],
                     default="attend",
                     help="attend: plain decode attention (the default line); append_attend: "

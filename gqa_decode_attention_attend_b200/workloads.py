@@ -134,19 +134,25 @@ def make(name, lengths: Sequence[int], num_heads, num_kv_heads, head_dim, dtype=
 
 # ---------------------------------------------------------------- named configurations
 
-CONFIG_NAMES = ("c1_fp32", "c2_bf16", "c3_split", "c4_ragged", "c5_long")
+CONFIG_NAMES = ("fp32_b1_n512", "bf16_b16_n4096", "bf16_b4_n32768", "bf16_b64_ragged16384",
+                "bf16_b1_n131072")
 
 CONFIG_TEXT = {
-    "c1_fp32": "fp32 GQA decode, batch 1, 8 Q / 4 KV heads, head_dim 64, cache len 512; "
-               "q,K,V iid U(-1,1); scale 1/sqrt(64); no carry",
-    "c2_bf16": "bf16 K/V, fp32 accumulation, bf16 q/out; batch 16, 32 Q / 8 KV heads, "
-               "head_dim 128, every sequence 4096 keys; q,K,V iid N(0,1)",
-    "c3_split": "bf16 split-KV stress; batch 4, 64 Q / 8 KV heads, head_dim 128, 32768 keys "
-                "each; q,K,V iid N(0,1); partial states merged by gqa_softmax_merge",
-    "c4_ragged": "ragged bf16 batch of 64 sequences, lengths uniform in [1,16384], 32 Q / 8 KV "
-                 "heads, head_dim 128; carry m~N(0,1), l~U(1,100), acc~N(0,1) folded in",
-    "c5_long": "bf16 long context; batch 1, 48 Q / 8 KV heads, head_dim 128, 131072 keys; "
-               "K 1.732*U(-1,1), V U(-1,1); planted key at depth 4096, amp 8",
+    "fp32_b1_n512":
+        "fp32 GQA decode, batch 1, 8 Q / 4 KV heads, head_dim 64, cache len 512; "
+        "q,K,V iid U(-1,1); scale 1/sqrt(64); no carry",
+    "bf16_b16_n4096":
+        "bf16 K/V, fp32 accumulation, bf16 q/out; batch 16, 32 Q / 8 KV heads, "
+        "head_dim 128, every sequence 4096 keys; q,K,V iid N(0,1)",
+    "bf16_b4_n32768":
+        "bf16 split-KV stress; batch 4, 64 Q / 8 KV heads, head_dim 128, 32768 keys "
+        "each; q,K,V iid N(0,1); partial states merged by gqa_softmax_merge",
+    "bf16_b64_ragged16384":
+        "ragged bf16 batch of 64 sequences, lengths uniform in [1,16384], 32 Q / 8 KV "
+        "heads, head_dim 128; carry m~N(0,1), l~U(1,100), acc~N(0,1) folded in",
+    "bf16_b1_n131072":
+        "bf16 long context; batch 1, 48 Q / 8 KV heads, head_dim 128, 131072 keys; "
+        "K 1.732*U(-1,1), V U(-1,1); planted key at depth 4096, amp 8",
 }
 
 
@@ -157,18 +163,18 @@ def ragged_lengths(batch, lo, hi, seed):
 
 def config(name):
     """The full-size named workloads (seeds 1..5)."""
-    if name == "c1_fp32":
+    if name == "fp32_b1_n512":
         w = make(name, [512], 8, 4, 64, dtype=torch.float32, dist="uniform", seed=1,
                  score_scale=1.0 / 8.0)
-    elif name == "c2_bf16":
+    elif name == "bf16_b16_n4096":
         w = make(name, [4096] * 16, 32, 8, 128, dist="normal", seed=2)
-    elif name == "c3_split":
+    elif name == "bf16_b4_n32768":
         w = make(name, [32768] * 4, 64, 8, 128, dist="normal", seed=3)
-    elif name == "c4_ragged":
+    elif name == "bf16_b64_ragged16384":
         gen = torch.Generator().manual_seed(4)
         lengths = torch.randint(1, 16385, (64,), generator=gen, dtype=torch.int64).tolist()
         w = make(name, lengths, 32, 8, 128, dist="normal", carry=True, gen=gen, seed=4)
-    elif name == "c5_long":
+    elif name == "bf16_b1_n131072":
         w = make(name, [131072], 48, 8, 128, dist="needle", seed=5,
                  needle=dict(amp=8.0, depth=4096))
     else:

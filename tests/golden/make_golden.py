@@ -3,7 +3,7 @@
 The pages this library follows print no worked numeric example, so every stored
 value here is the f64 oracle's, on seeded inputs from the shared generator:
 
-  c1_fp32_rows.json  config "fp32, batch 1, 8 Q / 4 KV heads, head_dim 64,
+  fp32_b1_n512_rows.json  config "fp32, batch 1, 8 Q / 4 KV heads, head_dim 64,
                      512 keys, U(-1,1), scale 1/8": all 8 output rows and their
                      (m, l) -- needle_core attn.rs `self_attn_incremental`
                      (GQA decode), USearch linear algebra § Attention (m, l).
@@ -26,11 +26,11 @@ from gqa_decode_attention_attend_b200 import workloads  # noqa: E402
 
 
 def c1_rows():
-    w = workloads.config("c1_fp32")
+    w = workloads.config("fp32_b1_n512")
     st = oracle.decode_attend(workloads.host_array(w.q), workloads.host_array(w.k),
                               workloads.host_array(w.v), w.offsets.numpy(), w.num_heads,
                               w.num_kv_heads, w.score_scale)
-    return dict(workload="c1_fp32", text=w.meta["text"], m=st.m.tolist(), l=st.l.tolist(),
+    return dict(workload="fp32_b1_n512", text=w.meta["text"], m=st.m.tolist(), l=st.l.tolist(),
                 out=st.out.tolist())
 
 
@@ -44,7 +44,7 @@ def needle_small():
 
 
 def main():
-    for name, fn in (("c1_fp32_rows.json", c1_rows), ("needle_small.json", needle_small)):
+    for name, fn in (("fp32_b1_n512_rows.json", c1_rows), ("needle_small.json", needle_small)):
         with open(os.path.join(HERE, name), "w") as f:
             json.dump(fn(), f, indent=1)
         print("wrote", name)

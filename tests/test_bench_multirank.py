@@ -26,7 +26,7 @@ def _worker(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=__import__("datetime").timedelta(seconds=60))
     try:
-        w = bench.rank_workload("c1_fp32", rank, world)
+        w = bench.rank_workload("fp32_b1_n512", rank, world)
         local_ms = 10.0 + 5.0 * rank                # rank 1 is the slow one
         ms = bench.max_over_ranks(local_ms, torch.device("cpu"), dist)
         digest = float(w.k.double().sum())
@@ -59,5 +59,5 @@ def test_two_gloo_ranks():
 
 def test_single_rank_identity():
     assert bench.max_over_ranks(3.5, torch.device("cpu"), None) == 3.5
-    w = bench.rank_workload("c1_fp32", 0, 1)
-    assert w.name == "c1_fp32" and w.kv_bytes() == 1 << 20
+    w = bench.rank_workload("fp32_b1_n512", 0, 1)
+    assert w.name == "fp32_b1_n512" and w.kv_bytes() == 1 << 20

@@ -26,7 +26,7 @@ def dev():
 
 # ------------------------------------------------------------------ full-size workloads
 
-@pytest.mark.parametrize("name", ["c1_fp32", "c2_bf16", "c5_long"])
+@pytest.mark.parametrize("name", ["fp32_b1_n512", "bf16_b16_n4096", "bf16_b1_n131072"])
 def test_full_config(dev, name):
     w = workloads.config(name)
     dw = gu.DevWorkload(w, dev)
@@ -34,7 +34,7 @@ def test_full_config(dev, name):
     ref = gu.oracle_state(w)
     gu.check_out(out, ref, w, what=f"{name} out")
     gu.check_state(st, ref, w, what=f"{name} state")
-    if name == "c5_long":
+    if name == "bf16_b1_n131072":
         # the planted key dominates channel 0 of the first head of every group
         hpk = w.num_heads // w.num_kv_heads
         for g in range(w.num_kv_heads):
@@ -43,18 +43,18 @@ def test_full_config(dev, name):
 
 
 def test_full_config_ragged_with_carry(dev):
-    w = workloads.config("c4_ragged")
+    w = workloads.config("bf16_b64_ragged16384")
     dw = gu.DevWorkload(w, dev)
     out, st = gu.run(dw, with_state=True)
     rows = list(range(0, w.batch * w.num_heads, 3))       # sampled query rows
     ref = gu.oracle_state(w, rows=rows)
-    gu.check_out(out, ref, w, rows=rows, what="c4 out")
-    gu.check_state(st, ref, w, rows=rows, what="c4 state")
+    gu.check_out(out, ref, w, rows=rows, what="ragged out")
+    gu.check_state(st, ref, w, rows=rows, what="ragged state")
 
 
 def test_full_config_split_pipeline(dev):
     """partials_out -> gqa_softmax_merge -> gqa_state_finalize on the split-KV stress workload."""
-    w = workloads.config("c3_split")
+    w = workloads.config("bf16_b4_n32768")
     dw = gu.DevWorkload(w, dev)
     rows = w.batch * w.num_heads
     _, S, chunk = gqa.gqa_decode_workspace_size(dw.q, dw.k, dw.v, dw.offsets, w.num_heads,
@@ -68,8 +68,8 @@ def test_full_config_split_pipeline(dev):
     gqa.gqa_softmax_merge(parts, merged_out=merged, want_out=False)
     out = gqa.gqa_state_finalize(merged, out_dtype=torch.bfloat16)
     ref = gu.oracle_state(w)
-    gu.check_out(out, ref, w, what="c3 finalize")
-    gu.check_state(merged, ref, w, what="c3 merged")
+    gu.check_out(out, ref, w, what="split pipeline finalize")
+    gu.check_state(merged, ref, w, what="split pipeline merged")
     # sampled partial states against the oracle over each split's own key range
     ranges = gu.split_ranges(w, chunk, S)
     pm, pl, pacc = parts.m.cpu().numpy(), parts.l.cpu().numpy(), parts.acc.cpu().numpy()
@@ -250,14 +250,14 @@ def test_stored_golden_values(dev):
     import json
     import os
     g = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
-                                    "c1_fp32_rows.json")))
-    w = workloads.config("c1_fp32")
+                                    "fp32_b1_n512_rows.json")))
+    w = workloads.config("fp32_b1_n512")
     dw = gu.DevWorkload(w, dev)
     out, st = gu.run(dw, with_state=True)
     ref = __import__("oracle").State(np.array(g["m"]), np.array(g["l"]), np.array(g["out"]) * np.array(g["l"])[:, None],
                                      np.array(g["out"]))
-    gu.check_out(out, ref, w, what="golden c1")
-    gu.assert_close(st.m.cpu().numpy(), ref.m, torch.float32, "golden c1 m")
+    gu.check_out(out, ref, w, what="golden fp32_b1_n512")
+    gu.assert_close(st.m.cpu().numpy(), ref.m, torch.float32, "golden fp32_b1_n512 m")
 
 
 def test_more_segments_than_the_fixed_ticket_region(dev):

@@ -59,14 +59,14 @@ def test_needle_structure():
 
 
 def test_config_sizes():
-    w = workloads.config("c1_fp32")
+    w = workloads.config("fp32_b1_n512")
     assert w.q.dtype == torch.float32 and w.kv_bytes() == 1 << 20
     lengths = workloads.ragged_lengths(64, 1, 16384, 4)
     assert len(lengths) == 64 and min(lengths) >= 1 and max(lengths) <= 16384
 
 
 def test_golden_c1_reproduced_by_oracle():
-    g = json.load(open(os.path.join(GOLDEN, "c1_fp32_rows.json")))
-    w = workloads.config("c1_fp32")
+    g = json.load(open(os.path.join(GOLDEN, "fp32_b1_n512_rows.json")))
+    w = workloads.config("fp32_b1_n512")
     st = oracle.decode_attend(w.q.numpy(), w.k.numpy(), w.v.numpy(), w.offsets.numpy(), 8, 4, 1 / 8)
     assert np.array_equal(st.out, np.array(g["out"])) and np.array_equal(st.m, np.array(g["m"]))
