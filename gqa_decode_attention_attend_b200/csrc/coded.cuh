@@ -66,7 +66,7 @@ __device__ __forceinline__ float block_weight_scale(float bound) {
 }
 
 // Decode attention straight from the codes, never rebuilding a row:
-//   q.K_j = sum_w c_jw (q . katom[i_jw])  -- a table qa[h][atom] of the CTA's
+//   q.K_j = sum_w c_jw (q . katom[i_jw])  -- a table qa[atom][h] of the CTA's
 //     query heads against every K atom, built once per CTA, then lookups;
 //   sum_j p_j V_j = sum_atom (sum_{j,w: i'_jw = atom} p_j c'_jw) vatom[atom]
 //     -- per-atom weights Wt[h][atom], multiplied by the V atoms once at the end.
@@ -103,7 +103,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   const int hpk = a.hpk, NA = c.n_atoms, W = c.words;
   const int slots = coded_code_slots(W);
   uint32_t* cbuf = dsm;                                        // [slots][2][W][NT] code ring
-  float* qa = reinterpret_cast<float*>(dsm + slots * 2 * W * NT);   // [hpk][NA] logits (base 2)
+  float* qa = reinterpret_cast<float*>(dsm + slots * 2 * W * NT);   // [NA][hpk] logits (base 2)
   float* Wt = qa + hpk * NA;                                   // [hpk][NA] value weights
   uint32_t* Wb = reinterpret_cast<uint32_t*>(Wt + hpk * NA);   // [hpk][NA] block weights, fixed point
 
@@ -215,7 +215,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
         }
       }
       const int at = a0 + lane / HMAX, h = lane % HMAX;
-      if (at < NA && h < hpk) qa[h * NA + at] = v[0] * a.scale_log2;
+      if (at < NA && h < hpk) qa[at * hpk + h] = v[0] * a.scale_log2;
     }
   }
   __syncthreads();
@@ -231,6 +231,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
     inv_prev[h] = 0.f;
   }
   bool bad = false;
+  const bool quad_heads = (hpk & 3) == 0;
 #pragma unroll 1
   for (int blk = 0; blk < nblk; ++blk) {
     const int kb = t.kbeg + blk * NT;
@@ -276,9 +277,24 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
           bad = true;
           continue;
         }
+        // an atom's logits of all heads sit side by side: 16-byte loads when
+        // heads_per_kv is a multiple of 4
+        const float* row = qa + idx * hpk;
+        if (quad_heads) {
 #pragma unroll
-        for (int h = 0; h < HMAX; ++h)
-          if (h < hpk) sc[h] = fmaf(cf, qa[h * NA + idx], sc[h]);
+          for (int q4 = 0; q4 < HMAX / 4; ++q4)
+            if (4 * q4 < hpk) {
+              const float4 t4 = *reinterpret_cast<const float4*>(row + 4 * q4);
+              sc[4 * q4] = fmaf(cf, t4.x, sc[4 * q4]);
+              sc[4 * q4 + 1] = fmaf(cf, t4.y, sc[4 * q4 + 1]);
+              sc[4 * q4 + 2] = fmaf(cf, t4.z, sc[4 * q4 + 2]);
+              sc[4 * q4 + 3] = fmaf(cf, t4.w, sc[4 * q4 + 3]);
+            }
+        } else {
+#pragma unroll
+          for (int h = 0; h < HMAX; ++h)
+            if (h < hpk) sc[h] = fmaf(cf, row[h], sc[h]);
+        }
       }
       const float bb = bias2(a, t, key);
 #pragma unroll
