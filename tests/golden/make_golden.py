@@ -25,7 +25,7 @@ import oracle  # noqa: E402
 from gqa_decode_attention_attend_b200 import workloads  # noqa: E402
 
 
-def c1_rows():
+def fp32_b1_n512_rows():
     w = workloads.config("fp32_b1_n512")
     st = oracle.decode_attend(workloads.host_array(w.q), workloads.host_array(w.k),
                               workloads.host_array(w.v), w.offsets.numpy(), w.num_heads,
@@ -44,7 +44,7 @@ def needle_small():
 
 
 def main():
-    for name, fn in (("fp32_b1_n512_rows.json", c1_rows), ("needle_small.json", needle_small)):
+    for name, fn in (("fp32_b1_n512_rows.json", fp32_b1_n512_rows), ("needle_small.json", needle_small)):
         with open(os.path.join(HERE, name), "w") as f:
             json.dump(fn(), f, indent=1)
         print("wrote", name)

@@ -65,7 +65,7 @@ def test_config_sizes():
     assert len(lengths) == 64 and min(lengths) >= 1 and max(lengths) <= 16384
 
 
-def test_golden_c1_reproduced_by_oracle():
+def test_golden_rows_reproduced_by_oracle():
     g = json.load(open(os.path.join(GOLDEN, "fp32_b1_n512_rows.json")))
     w = workloads.config("fp32_b1_n512")
     st = oracle.decode_attend(w.q.numpy(), w.k.numpy(), w.v.numpy(), w.offsets.numpy(), 8, 4, 1 / 8)
