@@ -242,8 +242,56 @@ def _default_workspace(device):
     return _default_ws[key]
 
 
+def _shape_error(what):
+    raise GqaError(GQA_ERR_SHAPE_MISMATCH, what)
+
+
+def _check_shapes(q, k, v, offsets, num_heads, num_kv_heads, carry, state_out, out, partials_out,
+                  num_splits, max_len, bias, kv_is_cache=True, check_out=True):
+    """The C ABI sees pointers only: check here that every tensor holds the
+    elements the call will touch, so a mismatched tensor is refused instead of
+    read or written past its end. Returns the split count to pass (the one
+    partials_out is laid out for, when num_splits is 0)."""
+    if offsets.dim() != 1 or offsets.numel() < 1 or str(offsets.dtype) != "torch.int32":
+        _shape_error("offsets must be a 1-D int32 tensor of batch + 1 entries")
+    B = offsets.numel() - 1
+    H = int(num_heads)
+    G = int(num_kv_heads) or H
+    D = q.shape[-1]
+    rows = B * H
+    if q.numel() != rows * D:
+        _shape_error(f"q holds {q.numel()} elements, expected batch*heads*head_dim = {rows * D}")
+    if kv_is_cache:
+        for name, t in (("k", k), ("v", v)):
+            if t.dim() != 3 or t.shape[1] != G or t.shape[2] != D:
+                _shape_error(f"{name} must be [max_len, {G}, {D}], got {list(t.shape)}")
+            if max_len is not None and int(max_len) > t.shape[0]:
+                _shape_error(f"max_len {int(max_len)} exceeds the {t.shape[0]} rows of {name}")
+    if check_out and out is not None and out.numel() != rows * D:
+        _shape_error(f"out holds {out.numel()} elements, expected {rows * D}")
+    for name, st in (("carry", carry), ("state_out", state_out)):
+        if st is not None and (st.m.numel() != rows or st.l.numel() != rows or st.acc.numel() != rows * D):
+            _shape_error(f"{name} must hold m, l [{rows}] and acc [{rows}, {D}]")
+    if partials_out is not None and rows > 0:
+        S, rem = divmod(partials_out.m.numel(), rows)
+        if rem or S < 1 or partials_out.l.numel() != rows * S or partials_out.acc.numel() != rows * S * D:
+            _shape_error(f"partials_out must hold m, l [{rows}, S] and acc [{rows}, S, {D}]")
+        if int(num_splits) == 0:
+            num_splits = S
+        elif int(num_splits) != S:
+            _shape_error(f"partials_out holds {S} splits per row, num_splits is {int(num_splits)}")
+    if bias is not None:
+        rows_needed = int(max_len) if max_len is not None else (k.shape[0] if kv_is_cache else 0)
+        if bias.numel() < rows_needed:
+            _shape_error(f"bias holds {bias.numel()} rows, the cache has {rows_needed}")
+    return int(num_splits)
+
+
 def _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out,
-            out_dtype, partials_out, num_splits, max_seq_len, max_len, bias=None, flags=0):
+            out_dtype, partials_out, num_splits, max_seq_len, max_len, bias=None, flags=0,
+            kv_is_cache=True, check_out=True):
+    num_splits = _check_shapes(q, k, v, offsets, num_heads, num_kv_heads, carry, state_out, out,
+                               partials_out, num_splits, max_len, bias, kv_is_cache, check_out)
     p = _CParams()
     p.struct_size = ctypes.sizeof(_CParams)
     p.q, p.q_dtype = _ptr(q), _dtype_code(q)
@@ -281,7 +329,8 @@ def gqa_decode_workspace_size(q, k, v, offsets, num_heads, num_kv_heads=0, *, sc
     # sizing never dereferences out; a one-element placeholder marks it as wanted
     placeholder = torch.empty(1, dtype=q.dtype, device=q.device) if want_out else None
     p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out,
-                placeholder, _dtype_code(q), partials_out, num_splits, max_seq_len, max_len)
+                placeholder, _dtype_code(q), partials_out, num_splits, max_seq_len, max_len,
+                check_out=False)
     nbytes = ctypes.c_size_t()
     ns = ctypes.c_int32()
     cl = ctypes.c_int32()
@@ -349,6 +398,9 @@ def gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_h
     are written), then attend with the new key included; see include/gqa_decode.h."""
     if k_new.dtype != k.dtype or v_new.dtype != k.dtype:
         raise GqaError(GQA_ERR_SHAPE_MISMATCH, "k_new/v_new must have the cache dtype")
+    rows_new = (offsets.numel() - 1) * k.shape[1] * k.shape[2]
+    if k_new.numel() != rows_new or v_new.numel() != rows_new:
+        _shape_error(f"k_new/v_new must be [batch, {k.shape[1]}, {k.shape[2]}]")
     return _attend_call("gqa_decode_append_attend", q, k, v, offsets, num_heads, num_kv_heads,
                         score_scale, carry, state_out, out, out_dtype, None, want_out, num_splits,
                         max_seq_len, max_len, workspace, stream, bias,
@@ -371,15 +423,23 @@ def gqa_decode_attend_coded(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_
     if out is not None:
         odt = _dtype_code(out)
     max_len = k_codes.shape[0]
+    G = int(num_kv_heads) or int(num_heads)
+    D = q.shape[-1]
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        if t.dim() != 3 or t.shape[0] != max_len or t.shape[1] != G or t.shape[2] != k_codes.shape[2]:
+            _shape_error(f"{name} must be [max_len, {G}, words], got {list(t.shape)}")
+    for name, t in (("k_atoms", k_atoms), ("v_atoms", v_atoms)):
+        if t.dim() != 2 or t.shape[1] != D or t.shape[0] != k_atoms.shape[0] or t.dtype != torch.float32:
+            _shape_error(f"{name} must be float32 [n_atoms, {D}], got {list(t.shape)}")
     p = _params(q, q, q, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
-                partials_out, num_splits, max_seq_len, max_len, bias, flags)
+                partials_out, num_splits, max_seq_len, max_len, bias, flags, kv_is_cache=False)
     p.k = p.v = None
     codes = _CCodes(_ptr(k_codes), _ptr(v_codes), k_codes.shape[-1], _ptr(k_atoms), _ptr(v_atoms),
                     k_atoms.shape[0])
     lib = load_library()
     # workspace sizing sees the code arrays in the caches' place
     pw = _params(q, q, q, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
-                 partials_out, num_splits, max_seq_len, max_len, bias, flags)
+                 partials_out, num_splits, max_seq_len, max_len, bias, flags, kv_is_cache=False)
     pw.k, pw.v = _ptr(k_codes), _ptr(v_codes)
     nbytes = ctypes.c_size_t()
     _check(lib.gqa_decode_workspace_size(ctypes.byref(pw), ctypes.byref(nbytes), None, None),

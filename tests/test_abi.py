@@ -150,3 +150,54 @@ def test_plan_degenerate():
         gqa.gqa_plan_splits(1, 0, 10, 10)
     with pytest.raises(gqa.GqaError):
         gqa.gqa_plan_splits(1, 1, 10, 10, 0, 2)
+
+
+_B, _H, _G, _D, _N = 2, 8, 2, 64, 10
+
+
+def _bad(name):
+    """One mismatched argument of a small decode call (CPU tensors)."""
+    import torch
+    rows = _B * _H
+    return {
+        "q": ("q", torch.zeros(_B, _H - 1, _D)),
+        "k_heads": ("k", torch.zeros(_B * _N, _G + 1, _D)),
+        "v_dim": ("v", torch.zeros(_B * _N, _G, _D // 2)),
+        "offsets_dtype": ("offsets", torch.tensor([0, _N, 2 * _N])),
+        "out": ("out", torch.zeros(rows * _D - 1)),
+        "carry": ("carry", gqa.State(torch.zeros(rows - 1), torch.zeros(rows - 1), torch.zeros(rows - 1, _D))),
+        "partials": ("partials_out", gqa.State(torch.zeros(rows * 3 + 1), torch.zeros(rows * 3 + 1),
+                                               torch.zeros(rows * 3 + 1, _D))),
+        "bias": ("bias", torch.zeros(_B * _N - 1)),
+        "max_len": ("max_len", 1000),
+    }[name]
+
+
+@pytest.mark.parametrize("name", ["q", "k_heads", "v_dim", "offsets_dtype", "out", "carry", "partials",
+                                  "bias", "max_len"])
+def test_binding_refuses_mismatched_tensors(name):
+    """The C ABI sees pointers only; the binding refuses tensors that do not
+    hold what the call would read or write, before anything runs."""
+    import torch
+    args = dict(q=torch.zeros(_B, _H, _D), k=torch.zeros(_B * _N, _G, _D), v=torch.zeros(_B * _N, _G, _D),
+                offsets=torch.tensor([0, _N, 2 * _N], dtype=torch.int32))
+    kw = {}
+    key, val = _bad(name)
+    (args if key in args else kw)[key] = val
+    with pytest.raises(gqa.GqaError) as e:
+        gqa.gqa_decode_attend(args["q"], args["k"], args["v"], args["offsets"], _H, _G, **kw)
+    assert e.value.status == gqa.GQA_ERR_SHAPE_MISMATCH
+
+
+def test_binding_takes_the_split_count_from_partials():
+    import torch
+    B, H, D = 2, 8, 64
+    parts = gqa.State(torch.zeros(B * H, 3), torch.zeros(B * H, 3), torch.zeros(B * H, 3, D))
+    n = gqa._check_shapes(torch.zeros(B, H, D), torch.zeros(20, 2, D), torch.zeros(20, 2, D),
+                          torch.tensor([0, 10, 20], dtype=torch.int32), H, 2, None, None, None, parts,
+                          0, None, None)
+    assert n == 3
+    with pytest.raises(gqa.GqaError):
+        gqa._check_shapes(torch.zeros(B, H, D), torch.zeros(20, 2, D), torch.zeros(20, 2, D),
+                          torch.tensor([0, 10, 20], dtype=torch.int32), H, 2, None, None, None, parts,
+                          4, None, None)
