@@ -247,11 +247,13 @@ def _shape_error(what):
 
 
 def _check_shapes(q, k, v, offsets, num_heads, num_kv_heads, carry, state_out, out, partials_out,
-                  num_splits, max_len, bias, kv_is_cache=True, check_out=True):
+                  num_splits, max_len, bias, kv_is_cache=True, sizing=False):
     """The C ABI sees pointers only: check here that every tensor holds the
     elements the call will touch, so a mismatched tensor is refused instead of
     read or written past its end. Returns the split count to pass (the one
-    partials_out is laid out for, when num_splits is 0)."""
+    partials_out is laid out for, when num_splits is 0). A sizing query
+    (sizing=True) only marks out / partials_out as wanted: their shapes are
+    not checked and the library's own split plan is reported."""
     if offsets.dim() != 1 or offsets.numel() < 1 or str(offsets.dtype) != "torch.int32":
         _shape_error("offsets must be a 1-D int32 tensor of batch + 1 entries")
     B = offsets.numel() - 1
@@ -267,12 +269,12 @@ def _check_shapes(q, k, v, offsets, num_heads, num_kv_heads, carry, state_out, o
                 _shape_error(f"{name} must be [max_len, {G}, {D}], got {list(t.shape)}")
             if max_len is not None and int(max_len) > t.shape[0]:
                 _shape_error(f"max_len {int(max_len)} exceeds the {t.shape[0]} rows of {name}")
-    if check_out and out is not None and out.numel() != rows * D:
+    if not sizing and out is not None and out.numel() != rows * D:
         _shape_error(f"out holds {out.numel()} elements, expected {rows * D}")
     for name, st in (("carry", carry), ("state_out", state_out)):
         if st is not None and (st.m.numel() != rows or st.l.numel() != rows or st.acc.numel() != rows * D):
             _shape_error(f"{name} must hold m, l [{rows}] and acc [{rows}, {D}]")
-    if partials_out is not None and rows > 0:
+    if partials_out is not None and rows > 0 and not sizing:
         S, rem = divmod(partials_out.m.numel(), rows)
         if rem or S < 1 or partials_out.l.numel() != rows * S or partials_out.acc.numel() != rows * S * D:
             _shape_error(f"partials_out must hold m, l [{rows}, S] and acc [{rows}, S, {D}]")
@@ -289,9 +291,9 @@ def _check_shapes(q, k, v, offsets, num_heads, num_kv_heads, carry, state_out, o
 
 def _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out,
             out_dtype, partials_out, num_splits, max_seq_len, max_len, bias=None, flags=0,
-            kv_is_cache=True, check_out=True):
+            kv_is_cache=True, sizing=False):
     num_splits = _check_shapes(q, k, v, offsets, num_heads, num_kv_heads, carry, state_out, out,
-                               partials_out, num_splits, max_len, bias, kv_is_cache, check_out)
+                               partials_out, num_splits, max_len, bias, kv_is_cache, sizing)
     p = _CParams()
     p.struct_size = ctypes.sizeof(_CParams)
     p.q, p.q_dtype = _ptr(q), _dtype_code(q)
@@ -330,7 +332,7 @@ def gqa_decode_workspace_size(q, k, v, offsets, num_heads, num_kv_heads=0, *, sc
     placeholder = torch.empty(1, dtype=q.dtype, device=q.device) if want_out else None
     p = _params(q, k, v, offsets, num_heads, num_kv_heads, score_scale, carry, state_out,
                 placeholder, _dtype_code(q), partials_out, num_splits, max_seq_len, max_len,
-                check_out=False)
+                sizing=True)
     nbytes = ctypes.c_size_t()
     ns = ctypes.c_int32()
     cl = ctypes.c_int32()

@@ -201,3 +201,15 @@ def test_binding_takes_the_split_count_from_partials():
         gqa._check_shapes(torch.zeros(B, H, D), torch.zeros(20, 2, D), torch.zeros(20, 2, D),
                           torch.tensor([0, 10, 20], dtype=torch.int32), H, 2, None, None, None, parts,
                           4, None, None)
+
+
+def test_sizing_query_keeps_the_library_plan():
+    """A sizing query only marks partials_out as wanted: a placeholder of any
+    shape neither fails nor fixes the split count."""
+    import torch
+    B, H, D = 2, 8, 64
+    one = gqa.State(torch.zeros(1), torch.zeros(1), torch.zeros(1, D))
+    n = gqa._check_shapes(torch.zeros(B, H, D), torch.zeros(20, 2, D), torch.zeros(20, 2, D),
+                          torch.tensor([0, 10, 20], dtype=torch.int32), H, 2, None, None,
+                          torch.zeros(1), one, 0, None, None, sizing=True)
+    assert n == 0
