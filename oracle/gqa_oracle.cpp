@@ -73,7 +73,11 @@ inline double f16_bits_to_f64(uint16_t bits) {
   const int f = bits & 0x3FF;
   double v;
   if (e == 0)
+#if ORACLE_MUTATION == 16
+    v = std::ldexp(static_cast<double>(f), -25);                // subnormals halved
+#else
     v = std::ldexp(static_cast<double>(f), -24);
+#endif
   else if (e == 31)
     v = f ? std::numeric_limits<double>::quiet_NaN() : std::numeric_limits<double>::infinity();
   else
@@ -141,6 +145,8 @@ void attend_one_row(const AttendArgs& a, int64_t row, int64_t r, std::vector<dou
     if (a.bias != nullptr) {
 #if ORACLE_MUTATION == 9
       s[t] = a.scale * (dot + static_cast<double>(a.bias[j]));   // bias inside the scale
+#elif ORACLE_MUTATION == 13
+      s[t] += static_cast<double>(a.bias[t]);                     // bias row of the sequence position
 #else
       s[t] += static_cast<double>(a.bias[j]);
 #endif
@@ -155,6 +161,9 @@ void attend_one_row(const AttendArgs& a, int64_t row, int64_t r, std::vector<dou
     lc = static_cast<double>(a.cl[row]);
     if (mc > m) m = mc;
   }
+#if ORACLE_MUTATION == 14
+  if (a.cl != nullptr && !has_carry && static_cast<double>(a.cm[row]) > m) m = a.cm[row];   // empty carry in the max
+#endif
 
   double* acc = a.oacc + r * D;
   for (int c = 0; c < D; ++c) acc[c] = 0.0;
@@ -181,7 +190,11 @@ void attend_one_row(const AttendArgs& a, int64_t row, int64_t r, std::vector<dou
       const double w = std::exp(mc - m);
 #endif
       l += lc * w;
+#if ORACLE_MUTATION == 12
+      for (int c = 0; c < D; ++c) acc[c] += static_cast<double>(a.cacc[row * D + c]);   // acc not rescaled
+#else
       for (int c = 0; c < D; ++c) acc[c] += static_cast<double>(a.cacc[row * D + c]) * w;
+#endif
     }
   }
 
@@ -281,7 +294,11 @@ int oracle_softmax_merge(const float* m, const float* l, const float* acc, int64
     double M = kNegInf;
     for (int i = 0; i < S; ++i) {
       const int64_t si = r * S + i;
+#if ORACLE_MUTATION == 15
+      if (static_cast<double>(m[si]) > M) M = m[si];                // empty states in the max
+#else
       if (l[si] != 0.0f && static_cast<double>(m[si]) > M) M = m[si];
+#endif
     }
     const bool has_carry = cl != nullptr && cl[r] != 0.0f;
     if (has_carry && static_cast<double>(cm[r]) > M) M = cm[r];

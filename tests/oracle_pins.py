@@ -267,6 +267,7 @@ def pin_merge_union(o):
     acc3 = np.concatenate([acc, np.full((n, 1, D), 7.0, np.float32)], 1)
     merged3 = o.merge(m3, l3, acc3)
     assert np.array_equal(merged3.out, merged.out), "empty state in merge"
+    assert np.array_equal(merged3.m, merged.m) and np.array_equal(merged3.l, merged.l), "empty state's m in merge"
     # the same union through the carry of attend
     sc = o.attend(q, kB, vB, offB, H, G, score_scale=0.9,
                   carry=(sa.m.astype(np.float32), sa.l.astype(np.float32), sa.acc.astype(np.float32)))
@@ -287,6 +288,7 @@ def pin_carry_identity(o):
     cacc = r.normal(0, 1, (n, D)).astype(np.float32)
     st = o.attend(q, k, v, off, H, G, carry=(cm, cl, cacc))
     assert np.array_equal(st.out, base.out) and np.array_equal(st.l, base.l), "empty carry"
+    assert np.array_equal(st.m, base.m), "empty carry's m"
     # the carry of an empty sequence passes through as acc/l
     cl = r.uniform(1, 2, n).astype(np.float32)
     st = o.attend(q[:1], k[:0], v[:0], np.array([0, 0], np.int32), H, G,

@@ -4,7 +4,10 @@ Every ORACLE_MUTATION build in oracle/gqa_oracle.cpp is a plausible slip: an
 interleaved head map, a dropped scale, a carry rescaled with the wrong sign, an
 output not divided by the partition, a transposed cache layout, partial states
 merged without rescaling, a dropped last key, keys used as values, a bias added
-before the scale, a top-k index one past a sequence's end accepted.
+before the scale, a top-k index one past a sequence's end accepted, the code
+word's fields swapped, a carry whose acc is not rescaled, a bias read by the
+key's position in its sequence, empty states (carry or merge input) raising the
+maximum, binary16 subnormals off by a factor of two.
 """
 import os
 
@@ -18,7 +21,9 @@ MUTATIONS = {1: "interleaved head map", 2: "scale dropped", 3: "carry sign flipp
              4: "not divided by partition", 5: "cache layout transposed",
              6: "merge without rescaling", 7: "last key dropped", 8: "keys used as values",
              9: "bias inside the scale", 10: "top-k admits one past the end",
-             11: "code word fields swapped"}
+             11: "code word fields swapped", 12: "carry acc not rescaled",
+             13: "bias indexed by sequence position", 14: "empty carry raises the maximum",
+             15: "merge counts empty states in the maximum", 16: "f16 subnormals halved"}
 
 
 @pytest.mark.parametrize("mutation", sorted(MUTATIONS), ids=lambda m: MUTATIONS[m])
