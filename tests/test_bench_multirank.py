@@ -61,3 +61,19 @@ def test_single_rank_identity():
     assert bench.max_over_ranks(3.5, torch.device("cpu"), None) == 3.5
     w = bench.rank_workload("fp32_b1_n512", 0, 1)
     assert w.name == "fp32_b1_n512" and w.kv_bytes() == 1 << 20
+
+
+def test_clock_summary_of_sampled_lines():
+    """The clocks record: median SM clock, the highest max clock, and every
+    throttle reason seen Active; malformed or unavailable samples are skipped."""
+    lines = [
+        "0, 1965, 1965, 700.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 1000.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, 10.0, 0x0, Not Active, Active, Not Active, Not Active",   # unavailable: skipped
+        "garbage line",
+    ]
+    c = bench.ClockSampler.summarize(lines)
+    assert c == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    assert bench.ClockSampler.summarize([]) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                                                "samples": 0}
