@@ -52,13 +52,16 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="bf16_b16_n4096")
-    ap.add_argument("--op", choices=["attend", "append_attend", "masked_attend", "coded_attend"],
+    ap.add_argument("--op", choices=["attend", "append_attend", "masked_attend", "coded_attend",
+                                     "split_pipeline"],
                     default="attend",
                     help="attend: plain decode attention (the default line); append_attend: "
                          "append the new token's K/V then attend; masked_attend: index rows -> "
                          "bias (gqa_topk_to_bias) then attend with it; coded_attend: the "
                          "same shape as a dictionary-coded cache (8 code words per row, 256 "
-                         "atoms), KV bytes = code bytes read")
+                         "atoms), KV bytes = code bytes read; split_pipeline: the three-call "
+                         "path (partial states, gqa_softmax_merge with the carry, "
+                         "gqa_state_finalize)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--e2e-steps", type=int, default=30)
@@ -292,6 +295,13 @@ def run_ours(args):
         run_op(*caches[i % len(caches)], st)
 
     flags = 0 if args.no_early_start else gqa.GQA_FLAG_EARLY_START
+    if args.op == "split_pipeline":
+        # the heuristic's split count (a sizing query), and the three calls' buffers
+        _, sp_splits, _ = gqa.gqa_decode_workspace_size(
+            q, caches[0][0], caches[0][1], offsets, H, G, score_scale=w.score_scale, want_out=False,
+            partials_out=gqa.State.empty(1, D, dev, (1,)), max_seq_len=w.max_seq_len)
+        sp_parts = gqa.State.empty(w.batch * H, D, dev, (sp_splits,))
+        sp_merged = gqa.State.empty(w.batch * H, D, dev)
 
     def run_op(k, v, st=None):
         st = st or stream
@@ -303,6 +313,12 @@ def run_ours(args):
             gqa.gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, H, G, score_scale=w.score_scale,
                                          carry=carry, out=out, max_seq_len=w.max_seq_len, workspace=ws,
                                          stream=st, flags=flags)
+        elif args.op == "split_pipeline":
+            gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, partials_out=sp_parts,
+                                  num_splits=sp_splits, max_seq_len=w.max_seq_len, workspace=ws, stream=st,
+                                  flags=flags)
+            gqa.gqa_softmax_merge(sp_parts, carry=carry, merged_out=sp_merged, want_out=False, stream=st)
+            gqa.gqa_state_finalize(sp_merged, out=out.view(w.batch * H, D), stream=st)
         elif args.op == "masked_attend":
             gqa.gqa_topk_to_bias(idx, offsets, w.total_rows, bias=bias, stream=st)
             gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
@@ -479,7 +495,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * (2 if args.op == "masked_attend" else 1),
+            "gpu_launches": args.steps * {"masked_attend": 2, "split_pipeline": 3}.get(args.op, 1),
             "launch_mode": ("eager" if args.eager else "cuda_graph_of_timed_steps") +
                            ("" if args.no_early_start else "+early_start"),
             "clocks": clocks,
