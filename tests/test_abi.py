@@ -213,3 +213,22 @@ def test_sizing_query_keeps_the_library_plan():
                           torch.tensor([0, 10, 20], dtype=torch.int32), H, 2, None, None,
                           torch.zeros(1), one, 0, None, None, sizing=True)
     assert n == 0
+
+
+def test_plan_invariants_over_random_shapes():
+    """For any batch the split plan is a valid cover of the longest sequence:
+    chunks of whole 64-row stages, ceil(N / chunk) of them, none empty."""
+    import random
+    rnd = random.Random(2024)
+    for _ in range(2000):
+        B = rnd.randint(1, 512)
+        G = rnd.choice([1, 2, 4, 8, 16])
+        N = rnd.randint(1, 300000)
+        full = B * N
+        total = rnd.choice([full, rnd.randint(1, full)])
+        sm = rnd.choice([1, 8, 132, 148, 160])
+        per_sm = rnd.choice([1, 2, 3])
+        chunk, splits = gqa.gqa_plan_splits(B, G, N, total, sm, per_sm)
+        assert chunk % 64 == 0 and chunk >= 64
+        assert splits >= 1 and splits == -(-N // chunk)
+        assert (splits - 1) * chunk < N <= splits * chunk
