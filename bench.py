@@ -3,11 +3,13 @@
 
 One step = one gqa_decode_attend call over the whole batch (one launch of the
 split-KV partition kernel, whose last CTA per sequence and KV head merges the
-splits and writes the output) on the 16-sequence bf16 workload: batch 16,
-32 Q / 8 KV heads, head_dim 128, 4096 cached keys per sequence, q/K/V iid
-N(0,1), bf16 output. Inputs are resident in HBM before the timed region; two
-copies of the 256 MiB cache are alternated so consecutive steps never read a
-cache the 126 MB L2 could still hold.
+splits and the carry and writes the output). The default workload is the
+largest one: a ragged bf16 batch of 64 sequences with lengths uniform in
+[1, 16384] (Arrow offsets), 32 Q / 8 KV heads, head_dim 128, q/K/V iid N(0,1),
+a per-query-row carry (m ~ N(0,1), l ~ U(1,100), acc ~ N(0,1)) folded in,
+bf16 output: ~2.15 GB of KV cache per step, resident in HBM before the timed
+region and far larger than the 126 MB L2. Smaller caches are duplicated and
+the copies alternated so no step reads a cache L2 could still hold.
 
 The K timed steps are captured once into a CUDA graph and replayed (the call
 allocates nothing and never synchronises), each launched with
@@ -17,11 +19,17 @@ reads); --eager and --no-early-start turn either off.
 Prints ONE JSON line (rank 0). `value` is the KV-cache bytes read per step,
 summed over ranks, divided by the max-over-ranks device time (GB/s); `e2e` is
 the same metric through the same public call when every step also copies its
-inputs from pinned host memory and its output back.
+inputs from pinned host memory and its output back. `targets` times, in the
+same run, the three long-context bf16 workloads that must each hold >= 70 % of
+the nominal 8 TB/s in KV bytes read: the 4 x 32768 split stress batch through
+the three-call path it names (partial states, gqa_softmax_merge with the
+carry, gqa_state_finalize), the ragged batch, and the 131072-key sequence;
+each with its step time back to back and as one isolated call after an L2
+flush, and its clock record.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--op OP] [--eager] [--no-early-start]
-                  [--no-cpu-baseline] [--quick]
+                  [--workload NAME] [--op OP] [--splits S] [--eager] [--no-early-start]
+                  [--no-cpu-baseline] [--no-targets] [--quick]
 
 --impl reference times the f64 CPU oracle (the library's reference
 implementation) on a bounded sample of the same workload, on rank 0 only.
@@ -29,7 +37,6 @@ implementation) on a bounded sample of the same workload, on rank 0 only.
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -51,10 +58,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="bf16_b16_n4096")
-    ap.add_argument("--op", choices=["attend", "append_attend", "masked_attend", "coded_attend",
-                                     "split_pipeline"],
-                    default="attend",
+    ap.add_argument("--workload", default="bf16_b64_ragged16384")
+    ap.add_argument("--op", choices=sorted(LAUNCHES), default="attend",
                     help="attend: plain decode attention (the default line); append_attend: "
                          "append the new token's K/V then attend; masked_attend: index rows -> "
                          "bias (gqa_topk_to_bias) then attend with it; coded_attend: the "
@@ -62,6 +67,10 @@ def parse():
                          "atoms), KV bytes = code bytes read; split_pipeline: the three-call "
                          "path (partial states, gqa_softmax_merge with the carry, "
                          "gqa_state_finalize)")
+    ap.add_argument("--splits", type=int, default=0,
+                    help="force this many splits per sequence (0: the library's heuristic)")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip timing the long-context workloads beside the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--e2e-steps", type=int, default=30)
@@ -241,11 +250,191 @@ def whole_job_gbs(kv_bytes_per_rank, world, ms_per_step_max):
 
 # ------------------------------------------------------------------ ours
 
+# Launches of the library's kernels per step of each op.
+LAUNCHES = {"attend": 1, "append_attend": 1, "masked_attend": 2, "coded_attend": 1, "split_pipeline": 3}
+
+# The long-context bf16 workloads that must hold >= 70 % of the nominal HBM
+# bandwidth in KV-cache bytes read, each timed through the call its
+# description names (the split stress workload through the three-call path).
+TARGETS = (("bf16_b4_n32768", "split_pipeline"), ("bf16_b64_ragged16384", "attend"),
+           ("bf16_b1_n131072", "attend"))
+
+
+class Op:
+    """One step of `op` on workload `w`, its inputs resident on `dev`.
+
+    attend: plain decode attention; append_attend: append the new token's K/V
+    then attend; masked_attend: index rows -> bias (gqa_topk_to_bias) then
+    attend with it; coded_attend: the same shape as a dictionary-coded cache
+    (8 code words per row, 256 atoms; KV bytes = code bytes read);
+    split_pipeline: the three-call path (partial states, gqa_softmax_merge with
+    the carry, gqa_state_finalize)."""
+
+    def __init__(self, w, op, dev, flags, num_splits=0):
+        import torch
+        import gqa_decode_attention_attend_b200 as gqa
+        self.gqa, self.w, self.op, self.flags, self.forced = gqa, w, op, flags, int(num_splits)
+        H, G, D = w.num_heads, w.num_kv_heads, w.head_dim
+        self.kv_bytes = w.kv_bytes()
+        self.q = w.q.to(dev)
+        self.offsets = w.offsets.to(dev)
+        # two cache copies, alternated step by step, unless one is already > 4x L2
+        self.caches = [(w.k.to(dev), w.v.to(dev))]
+        if self.kv_bytes < 4 * 126e6:
+            self.caches.append((self.caches[0][0].clone(), self.caches[0][1].clone()))
+        self.carry = gqa.State(*(t.to(dev) for t in w.carry)) if w.carry is not None else None
+        self.out = torch.empty(self.q.shape, dtype=self.q.dtype, device=dev)
+        self.ws = gqa.Workspace(dev)
+        gen = torch.Generator().manual_seed(77)
+        self.k_new = torch.randn((w.batch, G, D), generator=gen).to(w.k.dtype).to(dev)
+        self.v_new = torch.randn((w.batch, G, D), generator=gen).to(w.k.dtype).to(dev)
+        self.idx = torch.randint(-1, max(w.max_seq_len, 1), (w.batch, 512), generator=gen,
+                                 dtype=torch.int32).to(dev)
+        self.bias = torch.zeros(w.total_rows, dtype=torch.float32, device=dev)
+        self.kernel = ("gqa_partition_bf16_kernel" if w.k.dtype == torch.bfloat16
+                       else "gqa_partition_f32_kernel")
+        if op == "coded_attend":
+            words, n_atoms = 8, 256
+            cg = torch.Generator().manual_seed(78)
+            idx = torch.randint(0, n_atoms, (w.total_rows, G, words), generator=cg, dtype=torch.int64)
+            cf = torch.randn((w.total_rows, G, words), generator=cg).to(torch.float16).view(torch.int16)
+            code = ((idx << 16) | (cf.to(torch.int64) & 0xFFFF)).to(torch.int64)
+            code = torch.where(code >= 2**31, code - 2**32, code).to(torch.int32)
+            self.kcodes = code.to(dev).contiguous()
+            self.vcodes = torch.roll(code, 1, 0).to(dev).contiguous()
+            self.atoms = torch.nn.functional.normalize(torch.randn((n_atoms, D), generator=cg), dim=1).to(dev)
+            self.kv_bytes = 2 * self.kcodes.numel() * 4
+            self.kernel = "gqa_partition_coded_kernel"
+        # the split plan of the plain call, and the three-call path's buffers
+        self.S_ws, self.S, self.chunk = gqa.gqa_decode_workspace_size(
+            self.q, self.caches[0][0], self.caches[0][1], self.offsets, H, G, score_scale=w.score_scale,
+            want_out=True, num_splits=self.forced, max_seq_len=w.max_seq_len)
+        if op == "split_pipeline":
+            self.parts = gqa.State.empty(w.batch * H, D, dev, (self.S,))
+            self.merged = gqa.State.empty(w.batch * H, D, dev)
+        self.launches = LAUNCHES[op]
+
+    def run(self, i, st=None, flags=None):
+        gqa, w = self.gqa, self.w
+        H, G = w.num_heads, w.num_kv_heads
+        k, v = self.caches[i % len(self.caches)]
+        fl = self.flags if flags is None else flags
+        common = dict(score_scale=w.score_scale, max_seq_len=w.max_seq_len, workspace=self.ws, stream=st,
+                      flags=fl)
+        if self.op == "coded_attend":
+            gqa.gqa_decode_attend_coded(self.q, self.kcodes, self.vcodes, self.atoms, self.atoms, self.offsets,
+                                        H, G, carry=self.carry, out=self.out, num_splits=self.forced, **common)
+        elif self.op == "append_attend":
+            gqa.gqa_decode_append_attend(self.q, k, v, self.offsets, self.k_new, self.v_new, H, G,
+                                         carry=self.carry, out=self.out, num_splits=self.forced, **common)
+        elif self.op == "split_pipeline":
+            gqa.gqa_decode_attend(self.q, k, v, self.offsets, H, G, partials_out=self.parts,
+                                  num_splits=self.S, **common)
+            gqa.gqa_softmax_merge(self.parts, carry=self.carry, merged_out=self.merged, want_out=False,
+                                  stream=st)
+            gqa.gqa_state_finalize(self.merged, out=self.out.view(w.batch * H, w.head_dim), stream=st)
+        elif self.op == "masked_attend":
+            gqa.gqa_topk_to_bias(self.idx, self.offsets, w.total_rows, bias=self.bias, stream=st)
+            gqa.gqa_decode_attend(self.q, k, v, self.offsets, H, G, carry=self.carry, out=self.out,
+                                  bias=self.bias, num_splits=self.forced, **common)
+        else:
+            gqa.gqa_decode_attend(self.q, k, v, self.offsets, H, G, carry=self.carry, out=self.out,
+                                  num_splits=self.forced, **common)
+
+    def partials_only(self, i, st=None):
+        """The partition launch alone (partial states out, no merge)."""
+        gqa, w = self.gqa, self.w
+        if not hasattr(self, "parts_only"):
+            self.parts_only = gqa.State.empty(w.batch * w.num_heads, w.head_dim, self.q.device, (self.S,))
+        k, v = self.caches[i % len(self.caches)]
+        gqa.gqa_decode_attend(self.q, k, v, self.offsets, w.num_heads, w.num_kv_heads,
+                              score_scale=w.score_scale, partials_out=self.parts_only, num_splits=self.S,
+                              max_seq_len=w.max_seq_len, workspace=self.ws, stream=st)
+
+
+def time_steps(op, steps, warmup, eager):
+    """Device time (ms) of `steps` steps after `warmup` untimed ones, by CUDA
+    events on the launching stream. Unless `eager`, the K steps are captured
+    once into a CUDA graph and replayed (the calls allocate nothing and never
+    synchronise, so they capture as they are): the host's per-call marshalling
+    is then off the critical path, as in a serving loop. Returns (ms, replay)
+    where replay() re-runs the same timed work untimed."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        op.run(i)
+    torch.cuda.synchronize()
+    assert op.gqa.gqa_get_device_error(op.ws) == 0
+    graph = None
+    if not eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream()
+            for i in range(steps):
+                op.run(i, cap)
+        torch.cuda.synchronize()
+        graph.replay()                   # one untimed replay
+        torch.cuda.synchronize()
+
+    def replay():
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(steps):
+                op.run(i)
+
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1), replay, graph
+
+
+def time_isolated(op, reps=20):
+    """Median device time (ms) of one lone step: L2 flushed first (a 512 MiB
+    write), the GPU kept busy by a spin kernel while the host enqueues the call
+    (so no host gap is timed), plain stream order, no call before or after it
+    in flight."""
+    import torch
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=op.q.device)
+    times = []
+    for i in range(reps + 2):
+        flush.zero_()
+        torch.cuda._sleep(400000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        op.run(i, flags=0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(e0.elapsed_time(e1))
+    del flush
+    return statistics.median(times)
+
+
+def sampled(fn, sampler_gpu, min_s=1.5):
+    """Run fn() (timed work) under the clock sampler, then keep the same load
+    (fn's replay) for at least min_s seconds so the sampler sees it."""
+    import torch
+    sampler = ClockSampler(sampler_gpu)
+    sampler.start()
+    time.sleep(0.3)
+    t0 = time.perf_counter()
+    res = fn()
+    ms, replay = res[0], res[1]
+    while ms / 1e3 + (time.perf_counter() - t0) < min_s:
+        replay()
+        torch.cuda.synchronize()
+    return res, sampler.stop()
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
     import gqa_decode_attention_attend_b200 as gqa
-    from gqa_decode_attention_attend_b200 import workloads
 
     rank, world, local = dist_env()
     if world > 1:
@@ -253,203 +442,114 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    flags = 0 if args.no_early_start else gqa.GQA_FLAG_EARLY_START
+    peak, peak_src = measured_peaks()
 
     w = rank_workload(args.workload, rank, world)
-    H, G, D = w.num_heads, w.num_kv_heads, w.head_dim
-    kv_bytes = w.kv_bytes()
-    q = w.q.to(dev)
-    offsets = w.offsets.to(dev)
-    # two cache copies, alternated step by step (together > 2x L2)
-    caches = [(w.k.to(dev), w.v.to(dev))]
-    if kv_bytes < 4 * 126e6:
-        caches.append((caches[0][0].clone(), caches[0][1].clone()))
-    carry = gqa.State(*(t.to(dev) for t in w.carry)) if w.carry is not None else None
-    out = torch.empty(q.shape, dtype=q.dtype, device=dev)
-    ws = gqa.Workspace(dev)
-
-    gen = torch.Generator().manual_seed(77)
-    k_new = torch.randn((w.batch, G, D), generator=gen).to(w.k.dtype).to(dev)
-    v_new = torch.randn((w.batch, G, D), generator=gen).to(w.k.dtype).to(dev)
-    width = 512
-    idx = torch.randint(-1, max(w.max_seq_len, 1), (w.batch, width), generator=gen,
-                        dtype=torch.int32).to(dev)
-    bias = torch.zeros(w.total_rows, dtype=torch.float32, device=dev)
-
-    if args.op == "coded_attend":
-        # synthetic dictionary and codes of the workload's shape: 8 words per row
-        words, n_atoms = 8, 256
-        cg = torch.Generator().manual_seed(78)
-        idx = torch.randint(0, n_atoms, (w.total_rows, G, words), generator=cg, dtype=torch.int64)
-        cf = torch.randn((w.total_rows, G, words), generator=cg).to(torch.float16).view(torch.int16)
-        code = ((idx << 16) | (cf.to(torch.int64) & 0xFFFF)).to(torch.int64)
-        code = torch.where(code >= 2**31, code - 2**32, code).to(torch.int32)
-        kcodes = [code.to(dev).contiguous()]
-        vcodes = [torch.roll(code, 1, 0).to(dev).contiguous()]
-        atoms = torch.nn.functional.normalize(torch.randn((n_atoms, D), generator=cg), dim=1).to(dev)
-        kv_bytes = 2 * kcodes[0].numel() * 4
-
-    def step(i):
-        run_op(*caches[i % len(caches)])
-
-    def step_on(i, st):
-        run_op(*caches[i % len(caches)], st)
-
-    flags = 0 if args.no_early_start else gqa.GQA_FLAG_EARLY_START
-    if args.op == "split_pipeline":
-        # the heuristic's split count (a sizing query), and the three calls' buffers
-        _, sp_splits, _ = gqa.gqa_decode_workspace_size(
-            q, caches[0][0], caches[0][1], offsets, H, G, score_scale=w.score_scale, want_out=False,
-            partials_out=gqa.State.empty(1, D, dev, (1,)), max_seq_len=w.max_seq_len)
-        sp_parts = gqa.State.empty(w.batch * H, D, dev, (sp_splits,))
-        sp_merged = gqa.State.empty(w.batch * H, D, dev)
-
-    def run_op(k, v, st=None):
-        st = st or stream
-        if args.op == "coded_attend":
-            gqa.gqa_decode_attend_coded(q, kcodes[0], vcodes[0], atoms, atoms, offsets, H, G,
-                                        score_scale=w.score_scale, carry=carry, out=out,
-                                        max_seq_len=w.max_seq_len, workspace=ws, stream=st, flags=flags)
-        elif args.op == "append_attend":
-            gqa.gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, H, G, score_scale=w.score_scale,
-                                         carry=carry, out=out, max_seq_len=w.max_seq_len, workspace=ws,
-                                         stream=st, flags=flags)
-        elif args.op == "split_pipeline":
-            gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, partials_out=sp_parts,
-                                  num_splits=sp_splits, max_seq_len=w.max_seq_len, workspace=ws, stream=st,
-                                  flags=flags)
-            gqa.gqa_softmax_merge(sp_parts, carry=carry, merged_out=sp_merged, want_out=False, stream=st)
-            gqa.gqa_state_finalize(sp_merged, out=out.view(w.batch * H, D), stream=st)
-        elif args.op == "masked_attend":
-            gqa.gqa_topk_to_bias(idx, offsets, w.total_rows, bias=bias, stream=st)
-            gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
-                                  out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st,
-                                  bias=bias, flags=flags)
-        else:
-            gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, carry=carry,
-                                  out=out, max_seq_len=w.max_seq_len, workspace=ws, stream=st, flags=flags)
+    op = Op(w, args.op, dev, flags, args.splits)
+    kv_bytes = op.kv_bytes
+    H, D = w.num_heads, w.head_dim
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     args.warmup = max(args.warmup, 3)        # at least three untimed warm-up steps
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    assert gqa.gqa_get_device_error(ws) == 0
 
-    # The timed K steps are captured once into a CUDA graph (the calls allocate
-    # nothing and never synchronise, so they capture as-is) and replayed: the
-    # host's per-call marshalling is then off the critical path, as in a serving
-    # loop. --eager launches them one by one instead.
-    graph = None
-    if not args.eager:
+    def timed():
+        barrier()
+        res = time_steps(op, args.steps, args.warmup, args.eager)
         torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            cap_stream = torch.cuda.current_stream()
-            for i in range(args.steps):
-                step_on(i, cap_stream)
-        torch.cuda.synchronize()
-        graph.replay()                   # one untimed replay
-        torch.cuda.synchronize()
+        barrier()
+        return res
 
-    def timed_steps():
-        if graph is not None:
-            graph.replay()
-        else:
-            for i in range(args.steps):
-                step(i)
-
-    sampler = ClockSampler(local) if not args.quick else None
-    if sampler:
-        sampler.start()
-        time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    timed_steps()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    # keep the same load for at least ~1.5 s so the clock sampler sees it
-    extra_t0 = time.perf_counter()
-    i = 0
-    while sampler and ms_total / 1e3 + (time.perf_counter() - extra_t0) < 1.5:
-        timed_steps()
-        torch.cuda.synchronize()
-    clocks = sampler.stop() if sampler else None
-
+    if args.quick:
+        (ms_total, _, graph), clocks = timed(), None
+    else:
+        (ms_total, _, graph), clocks = sampled(timed, local)
+    del graph
     ms_max = max_over_ranks(ms_total, dev, dist if world > 1 else None)
     ms_per_step = ms_max / args.steps
     value = whole_job_gbs(kv_bytes, world, ms_per_step)
 
-    # ---- dominant kernel alone: the partition launch (partials-only call)
-    S_ws, S, chunk = gqa.gqa_decode_workspace_size(q, caches[0][0], caches[0][1], offsets, H, G,
-                                                   score_scale=w.score_scale, want_out=True,
-                                                   max_seq_len=w.max_seq_len)
-    parts = gqa.State.empty(w.batch * H, D, dev, (S,))
-
-    def part_only(i):
-        k, v = caches[i % len(caches)]
-        gqa.gqa_decode_attend(q, k, v, offsets, H, G, score_scale=w.score_scale, partials_out=parts,
-                              num_splits=S, max_seq_len=w.max_seq_len, workspace=ws, stream=stream)
-
+    # ---- the dominant kernel: one decode call is one launch of the partition
+    # kernel (the split merge runs inside it), so its launch duration is this
+    # rank's step time; the partials-only launch is reported beside it.
+    launch_ms = ms_total / args.steps
+    achieved = kv_bytes / (launch_ms / 1e3) / 1e9
     for i in range(5):
-        part_only(i)
+        op.partials_only(i)
     n_part = args.steps if args.quick else max(args.steps, 50)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(n_part):
-        part_only(i)
+        op.partials_only(i)
     e1.record(stream)
     torch.cuda.synchronize()
     part_ms = e0.elapsed_time(e1) / n_part
-    peak, peak_src = measured_peaks()
-    # A decode call is one launch of the partition kernel (the split merge runs
-    # inside it), so the dominant kernel's launch duration is the step time of
-    # this rank; the partials-only launch is reported beside it.
-    launch_ms = ms_total / args.steps
-    achieved = kv_bytes / (launch_ms / 1e3) / 1e9
+    iso_ms = None if args.quick else time_isolated(op)
 
     # ---- end to end: pinned host inputs -> device, call, output -> pinned host
-    hq = w.q.pin_memory()
-    hoff = w.offsets.pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    # the step's cache inputs: the raw K/V, or the code arrays for the coded op
-    if args.op == "coded_attend":
-        dev_cache = [kcodes[0], vcodes[0]]
-    else:
-        dev_cache = list(caches[0])
-    host_cache = [t.cpu().pin_memory() for t in dev_cache]
-    h2d = (hq.numel() * hq.element_size() + sum(t.numel() * t.element_size() for t in host_cache) +
-           hoff.numel() * 4)
-    d2h = hout.numel() * hout.element_size()
-
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        for d, h in zip(dev_cache, host_cache):
-            d.copy_(h, non_blocking=True)
-        offsets.copy_(hoff, non_blocking=True)
-        run_op(*caches[0])
-        hout.copy_(out, non_blocking=True)
-
     n_e2e = 0 if args.quick else args.e2e_steps
-    for _ in range(2 if n_e2e else 0):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    x0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
-    x1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / max(n_e2e, 1), dev, dist if world > 1 else None)
-    e2e_value = whole_job_gbs(kv_bytes, world, e2e_ms)
+    e2e = None
+    if n_e2e:
+        dev_in = [op.q, op.offsets]
+        dev_in += [op.kcodes, op.vcodes] if args.op == "coded_attend" else list(op.caches[0])
+        if op.carry is not None:
+            dev_in += [op.carry.m, op.carry.l, op.carry.acc]
+        host_in = [t.cpu().pin_memory() for t in dev_in]
+        hout = torch.empty(op.out.shape, dtype=op.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+            op.run(0)
+            hout.copy_(op.out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        x1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(x0.elapsed_time(x1) / n_e2e, dev, dist if world > 1 else None)
+        e2e = {"value": round(whole_job_gbs(kv_bytes, world, e2e_ms), 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        del host_in, hout
+
+    # ---- the long-context targets, each through the call its workload names
+    targets = None
+    if rank == 0 and world == 1 and not args.quick and not args.no_targets:
+        targets = {}
+        for name, top in TARGETS:
+            if name == w.name and top == args.op and not args.splits:
+                t_ms, t_iso, t_clk, t_op = launch_ms, iso_ms, clocks, op
+            else:
+                t_op = Op(rank_workload(name, 0, 1), top, dev, flags)
+                (t_total, _, g), t_clk = sampled(lambda: time_steps(t_op, args.steps, args.warmup,
+                                                                    args.eager), local)
+                del g
+                t_ms = t_total / args.steps
+                t_iso = time_isolated(t_op)
+            gbs = t_op.kv_bytes / (t_ms / 1e3) / 1e9
+            targets[name] = {
+                "op": top, "ms_per_step": t_ms, "gbs": round(gbs, 1),
+                "frac_of_measured": round(gbs / peak, 4), "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                "isolated_ms": t_iso,
+                "isolated_gbs": round(t_op.kv_bytes / (t_iso / 1e3) / 1e9, 1) if t_iso else None,
+                "num_splits": t_op.S, "chunk_len": t_op.chunk, "launches_per_step": t_op.launches,
+                "clocks": t_clk,
+            }
+            if t_op is not op:
+                del t_op
+                torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
@@ -473,33 +573,38 @@ def run_ours(args):
             "data": "synthetic (seeded, no dataset)",
             "config": {
                 "workload": w.name, "op": args.op, "text": w.meta.get("text", ""), "batch": w.batch,
-                "num_heads": H, "num_kv_heads": G, "head_dim": D, "seq_len": w.max_seq_len,
-                "kv_bytes_per_step": kv_bytes, "num_splits": S, "chunk_len": chunk,
-                "l2": f"inputs larger than L2: {len(caches)} cache copies of {kv_bytes / 2**20:.0f} MiB alternated",
+                "num_heads": H, "num_kv_heads": w.num_kv_heads, "head_dim": D, "seq_len": w.max_seq_len,
+                "total_rows": w.total_rows, "kv_bytes_per_step": kv_bytes, "num_splits": op.S,
+                "chunk_len": op.chunk,
+                "l2": (f"inputs larger than L2: {len(op.caches)} cache copies of "
+                       f"{kv_bytes / 2**20:.0f} MiB alternated" if len(op.caches) > 1 else
+                       f"inputs larger than L2: one {kv_bytes / 2**20:.0f} MiB cache, > 4x the 126 MB L2"),
                 "parallelism": f"replicas x{world} (independent batches, no collective)",
             },
             "queries_heads_per_s": w.batch * H * world / (ms_per_step / 1e3),
             "pct_of_nominal_8tbs": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
             "pct_of_measured_peak": round(100.0 * value / world / peak, 2),
             "roofline": {
-                "bound": "hbm",
-                "kernel": ("gqa_partition_coded_kernel" if args.op == "coded_attend" else
-                           "gqa_partition_bf16_kernel" if w.k.dtype == torch.bfloat16
-                           else "gqa_partition_f32_kernel"),
+                "bound": "hbm", "kernel": op.kernel,
                 "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_src, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name) if args.op == "attend" else None,
+                "frac": round(achieved / peak, 4),
+                "traffic": recorded_traffic(w.name) if args.op == "attend" and not args.splits else None,
                 "algorithmic_bytes_per_launch": kv_bytes, "launch_ms": launch_ms,
+                "isolated_launch_ms": iso_ms,
                 "partials_only_launch_ms": part_ms,
                 "partials_only_gbs": round(kv_bytes / (part_ms / 1e3) / 1e9, 1),
             },
             "cpu_baseline": cpu,
-            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * {"masked_attend": 2, "split_pipeline": 3}.get(args.op, 1),
+            "e2e": e2e,
+            "gpu_launches": args.steps * op.launches,
             "launch_mode": ("eager" if args.eager else "cuda_graph_of_timed_steps") +
                            ("" if args.no_early_start else "+early_start"),
             "clocks": clocks,
         }
+        if targets is not None:
+            line["targets"] = targets
+            line["targets_met_70pct_of_nominal"] = all(t["frac_of_nominal_8tbs"] >= 0.70
+                                                       for t in targets.values())
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -16,7 +16,6 @@ If the compiled library is missing the first call raises ``LibraryMissing``;
 there is no fallback implementation.
 """
 import ctypes
-import math
 import os
 
 __all__ = [
@@ -547,10 +546,6 @@ def gqa_plan_splits(batch, num_kv_heads, max_seq_len, total_rows, sm_count=148, 
                                           int(total_rows), int(sm_count), int(ctas_per_sm),
                                           ctypes.byref(c), ctypes.byref(s)), "gqa_plan_splits")
     return c.value, s.value
-
-
-def default_scale(head_dim):
-    return 1.0 / math.sqrt(head_dim)
 
 
 def gqa_decode_attend_static_workspace(q, k, v, offsets, num_heads, num_kv_heads=0, *, score_scale=0.0,

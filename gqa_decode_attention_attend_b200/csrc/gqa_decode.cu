@@ -810,23 +810,53 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB per GPU
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry point (the library links
+// no driver import), or null.
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
 std::mutex g_static_mu;
-void* g_static_scratch_addr[kMaxDevices] = {};
+struct StaticScratch {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+StaticScratch g_static_scratch_addr[kMaxDevices];
 
 // Device address of g_static_scratch on the current device. The host-side
-// symbol is only a stand-in, so the address is looked up once per device
-// (with that device current) and cached.
+// symbol is only a stand-in, so the address is looked up once per device, with
+// that device current, and cached together with its context: a new context
+// (the old one reset) has its own copy of the array and gets a new lookup.
 void* static_scratch_address(int dev) {
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr || get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_scratch_addr[dev] == nullptr) {
+  StaticScratch& e = g_static_scratch_addr[dev];
+  if (e.addr == nullptr || ctx != e.ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
-    g_static_scratch_addr[dev] = p;
+    if (get != nullptr && get(&ctx) != CUDA_SUCCESS) ctx = nullptr;   // the lookup may create it
+    e.addr = p;
+    e.ctx = ctx;
   }
-  return g_static_scratch_addr[dev];
+  return e.addr;
 }
 
 }  // namespace
@@ -845,13 +875,35 @@ extern "C" gqa_status gqa_decode_attend_static_workspace(const gqa_decode_params
   uint8_t* ws = static_cast<uint8_t*>(static_scratch_address(dev));
   if (ws == nullptr) return GQA_ERR_DEVICE;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  // The array keeps whatever the previous call left in it. The error word must
-  // start at zero; the segment tickets return to zero at the end of every
-  // completed call (and start at zero when the module loads); the partial
-  // states are written before they are read.
-  if (r.B > 0 && cudaMemsetAsync(ws, 0, sizeof(uint32_t), cs) != cudaSuccess) {
-    cudaGetLastError();
-    return GQA_ERR_DEVICE;
+  // The array keeps whatever the previous call left in it. The error word and
+  // the tickets of this call's segments (in the fixed region right after the
+  // header; larger batches use a region attend_impl clears itself) must start
+  // at zero, so both are cleared here, whatever an earlier call left; the
+  // partial states are written before they are read.
+  if (r.B > 0) {
+    size_t clear = sizeof(uint32_t);
+    if (r.want_merge && !r.clear_counters)
+      clear = kHeaderBytes + static_cast<size_t>(r.B) * r.G * sizeof(uint32_t);
+    if (cudaMemsetAsync(ws, 0, clear, cs) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_DEVICE;
+    }
   }
   return attend_impl(p, r, ws, cs);
 }
+
+#ifdef GQA_TEST_HOOKS
+// Test support, compiled only into the test copy of the library: fill the
+// static scratch's header and ticket region with the byte `fill` on `stream`,
+// as a call that stopped half way could have left it.
+extern "C" gqa_status gqa_test_soil_static_scratch(int32_t fill, gqa_stream_t stream) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GQA_ERR_DEVICE;
+  uint8_t* ws = static_cast<uint8_t*>(static_scratch_address(dev));
+  if (ws == nullptr) return GQA_ERR_DEVICE;
+  if (cudaMemsetAsync(ws, fill & 0xFF, kHeaderBytes + kTicketSlots * sizeof(uint32_t),
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GQA_ERR_DEVICE;
+  return GQA_OK;
+}
+#endif

@@ -368,13 +368,16 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
       accs[(warp * HP + hc + 1) * P + d + 8] = o[mt][nt][3] * f[nt][1];
     }
   ptx::named_barrier_sync(1, 32 * W);
-  if (*abort_flag) return;
-  store_partial<D, W, HP>(a, t, ms, ls, accs, ctid, 32 * W, nslots);
+  // A tile whose pipeline gave up (GQA_ERR_TIMEOUT is set) stores no partial
+  // state, but still takes its merge ticket, so that the segment's ticket
+  // counter returns to zero as after any other call.
+  const bool tile_aborted = *abort_flag != 0;
+  if (!tile_aborted) store_partial<D, W, HP>(a, t, ms, ls, accs, ctid, 32 * W, nslots);
   static_assert(C::kConsumerWarps == 4, "NamedSync128 spans the four consumer warps");
   if (a.merge) {
     ptx::named_barrier_sync(1, 32 * W);     // store_partial done with the ring scratch
     finish_segment<D, HP>(a, t, ctid, smM, smL, smC, smFlag, reinterpret_cast<float*>(smem),
-                          C::kWeightCap, bar_merge, NamedSync128{});
+                          C::kWeightCap, bar_merge, NamedSync128{}, tile_aborted);
   }
 }
 

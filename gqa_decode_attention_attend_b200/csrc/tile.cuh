@@ -487,10 +487,14 @@ __device__ __forceinline__ bool merge_segment_smem(const PartitionArgs& a, const
 
 // After the CTA's partial state is stored: take a ticket on the segment and,
 // if this CTA completed it, merge. All participating threads call this.
+// `aborted` (a tile whose pipeline gave up, with GQA_ERR_TIMEOUT already set):
+// the ticket is still taken, and the counter still reset by the last CTA, but
+// an aborted CTA merges nothing.
 template <int D, int HP, class Sync>
 __device__ __forceinline__ void finish_segment(const PartitionArgs& a, const Tile& t, int tid,
                                                float* smM, float* smL, float* smC, int* smFlag,
-                                               float* wts, int wcap, uint32_t bulk_bar, Sync sync) {
+                                               float* wts, int wcap, uint32_t bulk_bar, Sync sync,
+                                               bool aborted = false) {
   const int nsplit = live_splits(a, t);
   if (nsplit > 1) {
     // The barrier orders every thread's partial-state stores before thread 0's
@@ -503,12 +507,13 @@ __device__ __forceinline__ void finish_segment(const PartitionArgs& a, const Til
       const unsigned ticket = ptx::atomic_add_acq_rel_gpu(a.counters + seg, 1u);
       const int last = (ticket == static_cast<unsigned>(nsplit - 1));
       if (last) a.counters[seg] = 0u;   // every split has counted: reset for the next call
-      *smFlag = last;
+      *smFlag = last && !aborted;
     }
     sync();
     if (!*smFlag) return;
   } else {
     sync();                     // a single split: the CTA merges its own partial
+    if (aborted) return;
   }
   if (bulk_bar != 0u &&
       merge_segment_smem<D>(a, t, nsplit, tid, smM, smL, smC, reinterpret_cast<uint8_t*>(wts),

@@ -154,8 +154,10 @@ gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* by
                                      int32_t* num_splits, int32_t* chunk_len);
 
 /* Zero a workspace (its error word and its per-sequence merge tickets). Call
- * once after allocating a workspace, and again after a call reported
- * GQA_ERR_TIMEOUT (an abandoned call can leave tickets behind). */
+ * once after allocating a workspace. A call that reported GQA_ERR_TIMEOUT
+ * produced no valid output, but it still leaves the tickets at zero: every
+ * tile, including one whose pipeline wait gave up, takes its merge ticket and
+ * the last one resets the counter, so the workspace stays usable as it is. */
 gqa_status gqa_workspace_init(void* workspace, size_t workspace_bytes, gqa_stream_t stream);
 
 /* Decode attention with a mergeable online-softmax state ([attn.rs]
@@ -184,12 +186,16 @@ gqa_status gqa_decode_attend(const gqa_decode_params* params, gqa_stream_t strea
  *   - A call whose scratch need (gqa_decode_workspace_size) exceeds 16 MiB is
  *     refused with GQA_ERR_WORKSPACE.
  *   - The first call on each device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     that device current) and caches it with the CUDA context it belongs to;
+ *     make that first call before any stream capture. A later call under a
+ *     different context of that device (after cudaDeviceReset, say) looks the
+ *     address up again.
  *   - All calls share the one array and it keeps the last call's contents:
  *     calls that may run at the same time on the GPU (different streams, or
  *     different host threads) race on it and must be serialised by the caller.
- *   - The device error word is cleared at the start of each call and is not
+ *   - Each call starts by clearing, on the stream, the device error word and
+ *     the merge tickets it will use, so nothing an earlier call left behind
+ *     (an aborted call included) reaches its result. The error word is not
  *     readable through gqa_get_device_error; use gqa_decode_attend with a
  *     workspace to diagnose malformed offsets. */
 gqa_status gqa_decode_attend_static_workspace(const gqa_decode_params* params, gqa_stream_t stream);

@@ -260,6 +260,28 @@ def test_stored_golden_values(dev):
     gu.assert_close(st.m.cpu().numpy(), ref.m, torch.float32, "golden fp32_b1_n512 m")
 
 
+def test_stored_needle_trial(dev):
+    """The planted-key trial at 1024 keys (cortiq_engine NystromState example
+    `trial`: 6 Q / 2 KV heads, d 64, key planted at depth 64 with amplitude 8,
+    V[., 0] = 0 except the planted row) against the oracle's stored out[:, 0]
+    (tests/golden/needle_small.json): channel 0 of each output is the weight
+    the softmax gives the planted key, which dominates for each group's first
+    head (heads 0 and 3)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                    "needle_small.json")))
+    w = workloads.make(g["workload"], g["lengths"], g["heads"], g["kv_heads"], g["head_dim"], dist="needle",
+                       seed=g["seed"], needle=dict(amp=g["amp"], depth=g["depth"]))
+    dw = gu.DevWorkload(w, dev)
+    out, _ = gu.run(dw, out_dtype=torch.float32)
+    got0 = out.reshape(-1, g["head_dim"])[:, 0].cpu().numpy()
+    gu.assert_close(got0, np.array(g["out0"]), torch.bfloat16, "golden needle_small out[:, 0]")
+    hpk = g["heads"] // g["kv_heads"]
+    for h in range(0, g["heads"], hpk):
+        assert got0[h] > 0.5
+
+
 def test_more_segments_than_the_fixed_ticket_region(dev):
     """9000 sequences x 8 KV heads = 72000 (sequence, KV head) segments: the merge
     tickets then live in a region cleared on every call."""

@@ -70,3 +70,12 @@ def test_golden_rows_reproduced_by_oracle():
     w = workloads.config("fp32_b1_n512")
     st = oracle.decode_attend(w.q.numpy(), w.k.numpy(), w.v.numpy(), w.offsets.numpy(), 8, 4, 1 / 8)
     assert np.array_equal(st.out, np.array(g["out"])) and np.array_equal(st.m, np.array(g["m"]))
+
+
+def test_golden_needle_reproduced_by_oracle():
+    g = json.load(open(os.path.join(GOLDEN, "needle_small.json")))
+    w = workloads.make(g["workload"], g["lengths"], g["heads"], g["kv_heads"], g["head_dim"], dist="needle",
+                       seed=g["seed"], needle=dict(amp=g["amp"], depth=g["depth"]))
+    st = oracle.decode_attend(workloads.host_array(w.q), workloads.host_array(w.k), workloads.host_array(w.v),
+                              w.offsets.numpy(), g["heads"], g["kv_heads"])
+    assert np.array_equal(st.out[:, 0], np.array(g["out0"]))
