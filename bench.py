@@ -309,6 +309,10 @@ class Op:
         self.S_ws, self.S, self.chunk = gqa.gqa_decode_workspace_size(
             self.q, self.caches[0][0], self.caches[0][1], self.offsets, H, G, score_scale=w.score_scale,
             want_out=True, num_splits=self.forced, max_seq_len=w.max_seq_len)
+        if op == "coded_attend":
+            _, self.S, self.chunk = gqa.gqa_decode_coded_workspace_size(
+                self.q, self.kcodes, self.vcodes, self.atoms, self.atoms, self.offsets, H, G,
+                score_scale=w.score_scale, carry=self.carry, num_splits=self.forced, max_seq_len=w.max_seq_len)
         if op == "split_pipeline":
             self.parts = gqa.State.empty(w.batch * H, D, dev, (self.S,))
             self.merged = gqa.State.empty(w.batch * H, D, dev)

@@ -107,6 +107,9 @@ def load_library(path=None):
     lib.gqa_decode_attend.argtypes = [ctypes.POINTER(_CParams), sp]
     lib.gqa_decode_append_attend.argtypes = [ctypes.POINTER(_CParams), sp, sp, sp]
     lib.gqa_decode_attend_coded.argtypes = [ctypes.POINTER(_CParams), ctypes.POINTER(_CCodes), sp]
+    lib.gqa_decode_coded_workspace_size.argtypes = [ctypes.POINTER(_CParams), ctypes.POINTER(_CCodes),
+                                                    ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(i32),
+                                                    ctypes.POINTER(i32)]
     lib.gqa_topk_to_bias.argtypes = [sp, i32, i32, sp, i32, sp, sp, sp]
     lib.gqa_softmax_merge.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
     lib.gqa_softmax_merge_gathered.argtypes = [ps, i32, i32, i32, ps, ps, sp, i32, sp]
@@ -119,7 +122,7 @@ def load_library(path=None):
     for fn in ("gqa_decode_workspace_size", "gqa_workspace_init", "gqa_decode_attend", "gqa_softmax_merge",
                "gqa_state_finalize", "gqa_get_device_error", "gqa_plan_splits",
                "gqa_decode_append_attend", "gqa_topk_to_bias", "gqa_softmax_merge_gathered",
-               "gqa_decode_attend_coded"):
+               "gqa_decode_attend_coded", "gqa_decode_coded_workspace_size"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gqa_version.restype = ctypes.c_int32
     if path is None:
@@ -408,6 +411,45 @@ def gqa_decode_append_attend(q, k, v, offsets, k_new, v_new, num_heads, num_kv_h
                         extra=(ctypes.c_void_p(_ptr(k_new)), ctypes.c_void_p(_ptr(v_new))), flags=flags)
 
 
+def _coded_params(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_heads, num_kv_heads, score_scale,
+                  carry, state_out, out, odt, partials_out, num_splits, max_seq_len, bias, flags):
+    torch = _torch()
+    max_len = k_codes.shape[0]
+    G = int(num_kv_heads) or int(num_heads)
+    D = q.shape[-1]
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        if t.dim() != 3 or t.shape[0] != max_len or t.shape[1] != G or t.shape[2] != k_codes.shape[2]:
+            _shape_error(f"{name} must be [max_len, {G}, words], got {list(t.shape)}")
+    for name, t in (("k_atoms", k_atoms), ("v_atoms", v_atoms)):
+        if t.dim() != 2 or t.shape[1] != D or t.shape[0] != k_atoms.shape[0] or t.dtype != torch.float32:
+            _shape_error(f"{name} must be float32 [n_atoms, {D}], got {list(t.shape)}")
+    p = _params(q, q, q, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
+                partials_out, num_splits, max_seq_len, max_len, bias, flags, kv_is_cache=False)
+    p.k = p.v = None
+    codes = _CCodes(_ptr(k_codes), _ptr(v_codes), k_codes.shape[-1], _ptr(k_atoms), _ptr(v_atoms),
+                    k_atoms.shape[0])
+    return p, codes
+
+
+def gqa_decode_coded_workspace_size(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_heads, num_kv_heads=0,
+                                    *, score_scale=0.0, carry=None, state_out=None, want_out=True,
+                                    partials_out=None, num_splits=0, max_seq_len=0):
+    """(bytes, num_splits, chunk_len) of a gqa_decode_attend_coded call (the
+    coded kernel's own split plan)."""
+    torch = _torch()
+    # sizing never dereferences out; a one-element placeholder marks it as wanted
+    out = torch.empty(1, dtype=q.dtype, device=q.device) if want_out else None
+    p, codes = _coded_params(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_heads, num_kv_heads,
+                             score_scale, carry, state_out, None, _dtype_code(q), partials_out, num_splits,
+                             max_seq_len, None, 0)
+    p.out = _ptr(out)
+    nbytes, ns, cl = ctypes.c_size_t(), ctypes.c_int32(), ctypes.c_int32()
+    _check(load_library().gqa_decode_coded_workspace_size(ctypes.byref(p), ctypes.byref(codes),
+                                                          ctypes.byref(nbytes), ctypes.byref(ns),
+                                                          ctypes.byref(cl)), "gqa_decode_coded_workspace_size")
+    return nbytes.value, ns.value, cl.value
+
+
 def gqa_decode_attend_coded(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_heads, num_kv_heads=0,
                             *, score_scale=0.0, carry=None, state_out=None, out=None, out_dtype=None,
                             partials_out=None, want_out=None, num_splits=0, max_seq_len=0,
@@ -423,28 +465,13 @@ def gqa_decode_attend_coded(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_
         out = torch.empty(q.shape, dtype=_torch_dtype(odt), device=q.device)
     if out is not None:
         odt = _dtype_code(out)
-    max_len = k_codes.shape[0]
-    G = int(num_kv_heads) or int(num_heads)
-    D = q.shape[-1]
-    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
-        if t.dim() != 3 or t.shape[0] != max_len or t.shape[1] != G or t.shape[2] != k_codes.shape[2]:
-            _shape_error(f"{name} must be [max_len, {G}, words], got {list(t.shape)}")
-    for name, t in (("k_atoms", k_atoms), ("v_atoms", v_atoms)):
-        if t.dim() != 2 or t.shape[1] != D or t.shape[0] != k_atoms.shape[0] or t.dtype != torch.float32:
-            _shape_error(f"{name} must be float32 [n_atoms, {D}], got {list(t.shape)}")
-    p = _params(q, q, q, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
-                partials_out, num_splits, max_seq_len, max_len, bias, flags, kv_is_cache=False)
-    p.k = p.v = None
-    codes = _CCodes(_ptr(k_codes), _ptr(v_codes), k_codes.shape[-1], _ptr(k_atoms), _ptr(v_atoms),
-                    k_atoms.shape[0])
+    p, codes = _coded_params(q, k_codes, v_codes, k_atoms, v_atoms, offsets, num_heads, num_kv_heads,
+                             score_scale, carry, state_out, out, odt, partials_out, num_splits, max_seq_len,
+                             bias, flags)
     lib = load_library()
-    # workspace sizing sees the code arrays in the caches' place
-    pw = _params(q, q, q, offsets, num_heads, num_kv_heads, score_scale, carry, state_out, out, odt,
-                 partials_out, num_splits, max_seq_len, max_len, bias, flags, kv_is_cache=False)
-    pw.k, pw.v = _ptr(k_codes), _ptr(v_codes)
     nbytes = ctypes.c_size_t()
-    _check(lib.gqa_decode_workspace_size(ctypes.byref(pw), ctypes.byref(nbytes), None, None),
-           "gqa_decode_workspace_size")
+    _check(lib.gqa_decode_coded_workspace_size(ctypes.byref(p), ctypes.byref(codes), ctypes.byref(nbytes),
+                                               None, None), "gqa_decode_coded_workspace_size")
     ws = workspace or _default_workspace(q.device)
     ws.reserve(nbytes.value, stream)
     p.workspace = ws.ptr

@@ -29,19 +29,55 @@ struct CodedArgs {
 };
 
 constexpr int kMaxCodeWords = 16;
-constexpr int kCodedThreads = 256;     // one key per thread per block of keys
+constexpr int kCodedThreads = 512;     // threads of a coded-kernel CTA (one CTA per SM)
 // Largest heads_per_kv * n_atoms: three tables of that many words (logits,
-// value weights, the block's integer weights) in shared memory.
+// value weights, the round's integer weights) in shared memory.
 constexpr int kCodedMaxTableEntries = 12288;
+// Dynamic shared memory budget of the coded kernel (under the 227 KB a CTA may
+// hold, with room for its static shared memory).
+constexpr int kCodedSmemBudget = 212 * 1024;
+// 128 bytes of alignment slack, then a 256-byte header (mbarriers)
+constexpr int kCodedFixedBytes = 384;
+constexpr int kCodedMaxRoundKeys = 8192;
 
-// Code rows are prefetched into a ring of blocks: three slots (two blocks
-// ahead) up to 8 words per row, two slots (one block ahead) above.
-__host__ __device__ constexpr int coded_code_slots(int words) { return words <= 8 ? 3 : 2; }
-
-// Dynamic shared memory of the coded kernel: the code ring, then the three tables.
+// Shared memory plan of the coded kernel, the same on host and device. In
+// words, after the header:
+//   ring    P x W x 512: a thread's next P code rows (P = 4, 2 or 1, as many
+//           as fit with a round of 512 keys);
+//   round   KR x (V + hpk + 1): up to 8 words per row (V = W), the round's V
+//           code rows (above 8, V = 0: V rows pass through the ring twice
+//           instead); its logits (then weights) and |V coefficient| sums. KR
+//           keys, a multiple of 512, at most 8192, as many as fit. The round
+//           region also stages atom rows;
+//   tables  3 x hpk x n_atoms: logit table, value weights, round weights.
+__host__ __device__ constexpr int coded_vstore_words(int words) { return 0 * words; }
+__host__ __device__ constexpr int coded_table_words(int hpk, int n_atoms) { return 3 * hpk * n_atoms; }
+__host__ __device__ constexpr int coded_free_words() { return (kCodedSmemBudget - kCodedFixedBytes) / 4; }
+__host__ __device__ constexpr int coded_key_words(int words, int hpk) { return coded_vstore_words(words) + hpk + 1; }
+__host__ __device__ constexpr bool coded_ring_fits(int rows, int words, int hpk, int n_atoms) {
+  return rows * words * kCodedThreads + kCodedThreads * coded_key_words(words, hpk) +
+             coded_table_words(hpk, n_atoms) <=
+         coded_free_words();
+}
+__host__ __device__ constexpr int coded_ring_rows(int words, int hpk, int n_atoms) {
+  return coded_ring_fits(4, words, hpk, n_atoms)   ? 4
+         : coded_ring_fits(2, words, hpk, n_atoms) ? 2
+                                                   : 1;
+}
+__host__ __device__ constexpr int coded_round_keys_uncapped(int words, int hpk, int n_atoms) {
+  return (coded_free_words() - coded_ring_rows(words, hpk, n_atoms) * words * kCodedThreads -
+          coded_table_words(hpk, n_atoms)) / coded_key_words(words, hpk) / kCodedThreads * kCodedThreads;
+}
+__host__ __device__ constexpr int coded_round_keys(int words, int hpk, int n_atoms) {
+  return coded_round_keys_uncapped(words, hpk, n_atoms) > kCodedMaxRoundKeys
+             ? kCodedMaxRoundKeys
+             : coded_round_keys_uncapped(words, hpk, n_atoms);
+}
 __host__ __device__ constexpr size_t coded_smem_bytes(int words, int hpk, int n_atoms) {
-  return static_cast<size_t>(coded_code_slots(words)) * 2 * words * kCodedThreads * 4 +
-         static_cast<size_t>(3) * hpk * n_atoms * 4;
+  return kCodedFixedBytes +
+         4 * (static_cast<size_t>(coded_ring_rows(words, hpk, n_atoms)) * words * kCodedThreads +
+              static_cast<size_t>(coded_round_keys(words, hpk, n_atoms)) * coded_key_words(words, hpk) +
+              coded_table_words(hpk, n_atoms));
 }
 
 __device__ __forceinline__ float code_coeff(uint32_t word) {
@@ -65,47 +101,82 @@ __device__ __forceinline__ float block_weight_scale(float bound) {
   return __int_as_float((e + 127) << 23);                     // 2^e
 }
 
+// Per head h < hpk (unrolled up to HMAX): reduce v[h][w] over the NW warps
+// of the CTA with op, in a fixed order (lane w holds warp w's value, then a
+// butterfly), so every thread gets the same result.
+template <int HMAX, int NW, class Op>
+__device__ __forceinline__ void cta_reduce_heads(const float (*v)[NW], int hpk, int lane, float init,
+                                                 float (&out)[HMAX], Op op) {
+  static_assert(NW <= 32, "one lane per warp");
+#pragma unroll
+  for (int h = 0; h < HMAX; ++h) {
+    if (h >= hpk) break;
+    float x = lane < NW ? v[h][lane] : init;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x = op(x, __shfl_xor_sync(0xffffffffu, x, o));
+    out[h] = x;
+  }
+}
+
 // Decode attention straight from the codes, never rebuilding a row:
 //   q.K_j = sum_w c_jw (q . katom[i_jw])  -- a table qa[atom][h] of the CTA's
 //     query heads against every K atom, built once per CTA, then lookups;
 //   sum_j p_j V_j = sum_atom (sum_{j,w: i'_jw = atom} p_j c'_jw) vatom[atom]
 //     -- per-atom weights Wt[h][atom], multiplied by the V atoms once at the end.
-// Keys go in blocks of 256 (one per thread). Each thread copies the K and V
-// code rows of the blocks ahead into shared memory (cp.async, its own slots)
-// while the current block runs. Per block: logits by table lookup, the
-// block's maximum per head (barrier), the weights p, the bound on each head's
-// weight sums (barrier), then every weight p * c is added to an integer table
-// Wb in fixed point scaled to that bound (32-bit shared atomics, which B200
-// executes several times faster than float ones, and whose sums do not
-// depend on their order; barrier); at the next block's start Wb is folded
-// into the float table Wt, rescaled to the new running maximum. The partition
-// l is kept per thread and reduced once. So the coded kernel's results are
-// bit-reproducible. The logit table is built by whole warps, lanes across D
-// (coalesced atom rows), with a warp reduce-scatter of the partial dot
-// products; the V atoms are applied by whole warps the same way (lanes across
-// D, no cross-lane sums). Same tiles, partial states and
-// fused merge as the other partition kernels. Two CTAs per SM for the usual
-// table sizes (registers capped at 128), as the split plan assumes.
-// MW: a compile-time bound on the words per row (4, 8 or 16) for the per-key loops.
+// One CTA of 512 threads per SM. Atom rows come into shared memory by TMA bulk
+// copies, two chunks in flight, for the logit table (warps take atoms, lanes
+// across D, a warp reduce-scatter sums the partial dot products) and for the
+// value epilogue (threads own 4 columns of one head for a share of the atoms,
+// then the shares add in a fixed order).
+// Keys go in rounds of KR (a multiple of 512); thread tid takes keys tid, tid
+// + 512, ... of a round. Its K code rows pass through its own P-row ring and
+// its V code rows land in its own slots of the round's V store (cp.async, the
+// next round's copies issued as soon as the thread is done with the current
+// one's rows, so they run across the barriers; no thread touches another's
+// slots); rows above 8 words, whose V store would not fit beside the largest
+// tables, instead pass through the ring again for passes B and C. Per round,
+// three passes and two barriers:
+//   A. logits by table lookups into the round's logit store, each key's sum of
+//      |V coefficient| from its V row, the warps' maxima per head -> barrier;
+//   B. the new running maximum; the last round's integer weights folded into
+//      Wt, both rescaled to it; each key's weights p (over its logits in the
+//      store), the partition, and per head the bound sum_j p_j sum_w |c'_jw|
+//      on any atom's weight sum -> barrier;
+//   C. every weight p * c' added to the integer table Wb in fixed point,
+//      scaled by a power of two that keeps the bound below 2^30 (32-bit
+//      shared atomics, which B200 runs several times faster than float ones,
+//      and whose sums do not depend on their order).
+// Cross-warp maxima and sums go through a fixed-order lane butterfly, so the
+// results are bit-reproducible. A segment with one split (the tile is the
+// whole sequence) folds the carry and writes out / state_out directly; others
+// go through the same partial states and fused merge as the other partition
+// kernels. MW: a compile-time bound on the words per row (4, 8 or 16).
 template <int D, int HMAX, int MW>
-__global__ void __launch_bounds__(kCodedThreads, 2)
+__global__ void __launch_bounds__(kCodedThreads, 1)
 gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   static_assert(MW == 4 || MW == 8 || MW == 16, "words bound 4, 8 or 16");
   constexpr int NT = kCodedThreads, NW = NT / 32, E = D / 32;
-  extern __shared__ __align__(16) uint32_t dsm[];
-  __shared__ __align__(16) float qs[HMAX * D];
-  __shared__ float accb[HMAX * D];
-  __shared__ float red[NW][HMAX];        // per warp: maxima per head (then partitions)
-  __shared__ float red2[NW][HMAX];       // per warp: weight bounds per head
+  constexpr bool VST = MW < 0;           // V rows kept in the round's store (else streamed twice)
+  extern __shared__ uint8_t dsm_raw[];
+  uint32_t* dsm = reinterpret_cast<uint32_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
+  __shared__ float red[HMAX][NW];        // per head, per warp: maxima (then partitions)
+  __shared__ float red2[2][HMAX][NW];    // per head, per warp: weight bounds, by round parity
   __shared__ float smM[16], smL[16], smC[16];
+  __shared__ float hM[16], hL[16];       // per head: base-2 running maximum, partition
   __shared__ int smFlag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hpk = a.hpk, NA = c.n_atoms, W = c.words;
-  const int slots = coded_code_slots(W);
-  uint32_t* cbuf = dsm;                                        // [slots][2][W][NT] code ring
-  float* qa = reinterpret_cast<float*>(dsm + slots * 2 * W * NT);   // [NA][hpk] logits (base 2)
+  const int P = coded_ring_rows(W, hpk, NA);
+  const int KR = coded_round_keys(W, hpk, NA);
+  const uint32_t bar0 = ptx::smem_u32(dsm);                    // atom copies into buffer 0 / 1
+  const uint32_t bar1 = bar0 + 8;
+  uint32_t* ring = dsm + 64;                                   // [P][W or W/4 quads][NT] K rows
+  uint32_t* vst = ring + P * W * NT;                           // [W or W/4 quads][KR] V rows (VST)
+  float* lg = reinterpret_cast<float*>(vst + (VST ? KR * W : 0));   // [KR][hpk] logits, then weights
+  float* cs = lg + KR * hpk;                                   // [KR] sums of |V coefficient|
+  float* qa = cs + KR;                                         // [NA][hpk] logits (base 2)
   float* Wt = qa + hpk * NA;                                   // [hpk][NA] value weights
-  uint32_t* Wb = reinterpret_cast<uint32_t*>(Wt + hpk * NA);   // [hpk][NA] block weights, fixed point
+  uint32_t* Wb = reinterpret_cast<uint32_t*>(Wt + hpk * NA);   // [hpk][NA] round weights, fixed point
 
   const Tile t = tile_of(a, blockIdx.x);
   ptx::grid_dependency_wait();
@@ -115,40 +186,35 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       merge_segment<D, HMAX>(a, t, 0, tid, smM, smL, smC, qa, hpk * NA, NamedSync128{});
     return;
   }
-
-  // This thread's code rows of block number `blk` (keys kbeg + 256 blk ..) go
-  // to its own slots of ring slot blk % slots: K then V, as 16-byte quads
-  // (quad-major, then thread) when the row is a multiple of 4 words, else word
-  // by word (word-major). One commit group per block, empty past the tile.
+  if (tid == 0) {
+    ptx::mbar_init(bar0, 1);
+    ptx::mbar_init(bar1, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
   const bool quads = (W & 3) == 0;
-  const uint32_t cbuf_u32 = ptx::smem_u32(cbuf);
-  const int nblk = (t.kend - t.kbeg + NT - 1) / NT;
-  auto stage_codes = [&](int blk) {
-    const int key = t.kbeg + blk * NT + tid;
-    if (blk < nblk && key < t.kend) {
-      const size_t row = ((static_cast<size_t>(t.o0) + key) * a.G + t.g) * W;
-      const uint32_t base = cbuf_u32 + (blk - (blk / slots) * slots) * 2 * W * NT * 4;
-      if (quads) {
-        for (int q = 0; q < W / 4; ++q) {
-          ptx::cp_async_16(base + ((0 * (W / 4) + q) * NT + tid) * 16, c.k_codes + row + 4 * q);
-          ptx::cp_async_16(base + ((1 * (W / 4) + q) * NT + tid) * 16, c.v_codes + row + 4 * q);
-        }
-      } else {
-        for (int w = 0; w < W; ++w) {
-          ptx::cp_async_4(base + ((0 * W + w) * NT + tid) * 4, c.k_codes + row + w);
-          ptx::cp_async_4(base + ((1 * W + w) * NT + tid) * 4, c.v_codes + row + w);
-        }
-      }
+  const int nround = (t.kend - t.kbeg + KR - 1) / KR;
+  const size_t row_stride = static_cast<size_t>(a.G) * W;
+  const uint32_t* kbase = c.k_codes + (static_cast<size_t>(t.o0) * a.G + t.g) * W;
+  const uint32_t* vbase = c.v_codes + (static_cast<size_t>(t.o0) * a.G + t.g) * W;
+  auto round_keys = [&](int rd) { return min(KR, t.kend - t.kbeg - rd * KR); };
+  auto rows_of = [&](int nk) { return nk > tid ? (nk - tid + NT - 1) / NT : 0; };
+
+  // ---- code rows
+  const uint32_t ring_u32 = ptx::smem_u32(ring), vst_u32 = ptx::smem_u32(vst);
+  auto copy_row = [&](uint32_t dst, int step, const uint32_t* src) {   // step: bytes between quads / words
+    if (quads) {
+      for (int q = 0; q < W / 4; ++q) ptx::cp_async_16(dst + q * step, src + 4 * q);
+    } else {
+      for (int w = 0; w < W; ++w) ptx::cp_async_4(dst + w * step, src + w);
     }
-    ptx::cp_async_commit();
   };
-  // this thread's K (kv = 0) or V (kv = 1) code row of a block out of its ring slot
-  auto load_row = [&](const uint32_t* sl, int kv, uint32_t (&r)[MW]) {
+  auto read_row = [&](const uint32_t* base, int stride, uint32_t (&r)[MW]) {   // stride: quads / words
     if (quads) {
 #pragma unroll
       for (int q = 0; q < MW / 4; ++q) {
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (4 * q < W) v = reinterpret_cast<const uint4*>(sl)[(kv * (W / 4) + q) * NT + tid];
+        if (4 * q < W) v = reinterpret_cast<const uint4*>(base)[q * stride];
         r[4 * q] = v.x;
         r[4 * q + 1] = v.y;
         r[4 * q + 2] = v.z;
@@ -156,225 +222,385 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       }
     } else {
 #pragma unroll
-      for (int w = 0; w < MW; ++w) r[w] = w < W ? sl[(kv * W + w) * NT + tid] : 0u;
+      for (int w = 0; w < MW; ++w) r[w] = w < W ? base[w * stride] : 0u;
     }
   };
-  for (int blk = 0; blk < slots - 1; ++blk) stage_codes(blk);
+  // Row i of this thread's keys of `base` in the round starting at kb into ring
+  // slot i % P (one commit group, empty past its rows)
+  auto issue_row = [&](const uint32_t* base, int kb, int mine, int i) {
+    if (i < mine) {
+      const int sl = i % P;
+      copy_row(ring_u32 + (quads ? (sl * (W / 4) * NT + tid) * 16 : (sl * W * NT + tid) * 4),
+               quads ? NT * 16 : NT * 4, base + static_cast<size_t>(kb + tid + i * NT) * row_stride);
+    }
+    ptx::cp_async_commit();
+  };
+  auto prime = [&](const uint32_t* base, int kb, int mine) {
+    for (int i = 0; i < P; ++i) issue_row(base, kb, mine, i);
+  };
+  auto wait_ring = [&] {             // the oldest of the P rows in flight has landed
+    if (P >= 4)
+      ptx::cp_async_wait_group<3>();
+    else if (P == 2)
+      ptx::cp_async_wait_group<1>();
+    else
+      ptx::cp_async_wait_group<0>();
+  };
+  auto ring_row = [&](int i, uint32_t (&r)[MW]) {
+    const int sl = i % P;
+    read_row(ring + (quads ? (sl * (W / 4) * NT + tid) * 4 : sl * W * NT + tid), NT, r);
+  };
+  // A round's copies: with the V store, this thread's V rows (one group,
+  // older than every K row of the round, so a K row that has landed means they
+  // have too); then its first P K rows.
+  auto start_round = [&](int rd) {
+    const int kb = t.kbeg + rd * KR, nk = round_keys(rd), mine = rows_of(nk);
+    if (VST) {
+      for (int i = 0; i < mine; ++i) {
+        const int j = tid + i * NT;
+        copy_row(vst_u32 + (quads ? j * 16 : j * 4), quads ? KR * 16 : KR * 4,
+                 vbase + static_cast<size_t>(kb + j) * row_stride);
+      }
+      ptx::cp_async_commit();
+    }
+    prime(kbase, kb, mine);
+  };
+  if (nround > 0) start_round(0);
 
-  // query rows of the group
-  const size_t qrow = static_cast<size_t>(t.b) * a.H + static_cast<size_t>(t.g) * hpk;
-  for (int i = tid; i < hpk * D; i += NT) {
-    qs[i] = c.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qrow * D + i])
-                     : static_cast<const float*>(a.q)[qrow * D + i];
-    accb[i] = 0.f;
-  }
+  // ---- atom rows: chunks of `chunk` atoms through two buffers in the logit
+  // store region, by bulk copies completing on bar0 / bar1. A chunk's copy is
+  // issued once every thread is done with the buffer (a barrier, and a proxy
+  // fence for the generic accesses before it); a wait that gives up flags
+  // GQA_ERR_TIMEOUT, lets the copy land (bounded) and turns `ok` false in every
+  // thread (a vote).
+  uint32_t phase0 = 0u, phase1 = 0u;
+  float* abuf = lg;
+  const int region = KR * (hpk + 1);                  // words of lg + cs (free outside rounds)
+  auto issue_atoms = [&](const float* atoms, int a0, int n, int b, float* base) {
+    if (tid == 0 && n > 0) {
+      const uint32_t bb = b ? bar1 : bar0;
+      ptx::mbar_arrive_expect_tx(bb, static_cast<uint32_t>(n) * D * 4);
+      ptx::bulk_load_1d(ptx::smem_u32(base), atoms + static_cast<size_t>(a0) * D, static_cast<uint32_t>(n) * D * 4, bb);
+    }
+  };
+  auto wait_atoms = [&](int b) -> bool {
+    const uint32_t bb = b ? bar1 : bar0;
+    const uint32_t ph = b ? phase1 : phase0;
+    const bool landed = ptx::mbar_wait_bounded(bb, ph, nullptr, kWaitLimitNs);
+    const bool all = __syncthreads_and(landed) != 0;
+    if (!all) {
+      if (tid == 0) atomicOr(a.err, kErrTimeout);
+      if (!landed) ptx::mbar_wait_bounded(bb, ph, nullptr, kWaitLimitNs);
+    }
+    if (b)
+      phase1 ^= 1u;
+    else
+      phase0 ^= 1u;
+    return all;
+  };
+  // Run body(chunk start, count, rows) over all atoms of `atoms`, two chunks in flight.
+  bool ok = true;
+  auto over_atoms = [&](const float* atoms, float* base, int words, auto&& body) {
+    const int chunk = words / 2 / D;                   // atoms per buffer
+    float* const buf1 = base + static_cast<size_t>(chunk) * D;
+    const int nchunk = (NA + chunk - 1) / chunk;
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
+    issue_atoms(atoms, 0, min(chunk, NA), 0, base);
+    if (nchunk > 1) issue_atoms(atoms, chunk, min(chunk, NA - chunk), 1, buf1);
+    for (int k = 0; k < nchunk && ok; ++k) {
+      const int b = k & 1;
+      float* const bufk = b ? buf1 : base;
+      ok = wait_atoms(b);
+      if (!ok) break;
+      body(k * chunk, min(chunk, NA - k * chunk), bufk);
+      if (k + 2 < nchunk) {
+        ptx::fence_proxy_async_smem();
+        __syncthreads();                               // buffer b read by everyone
+        issue_atoms(atoms, (k + 2) * chunk, min(chunk, NA - (k + 2) * chunk), b, bufk);
+      }
+    }
+  };
+
   for (int i = tid; i < hpk * NA; i += NT) {
     Wt[i] = 0.f;
     Wb[i] = 0u;
   }
-  __syncthreads();
-  // the logit table: a warp takes A = 32 / HMAX atoms per pass, lanes across D
-  // (coalesced rows, two passes of loads in flight). Each lane's A x HMAX
-  // partial dot products are summed across the warp by a reduce-scatter: at
-  // each of 5 steps a lane keeps half of its values and adds the other half
-  // from the lane `off` away, so lane L ends with atom L / HMAX, head L % HMAX.
+  // the logit table, HT heads at a time (at most 8, for registers): a warp
+  // takes A = 32 / HT atoms per pass, lanes across D (the rows out of shared
+  // memory). Each lane's A x HT partial dot products are summed across the
+  // warp by a reduce-scatter: at each of 5 steps a lane keeps half of its
+  // values and adds the other half from the lane `off` away, so lane L ends
+  // with atom L / HT, head L % HT of the pass.
   {
-    constexpr int A = 32 / HMAX;
-    float qreg[HMAX][E];
+    constexpr int HT = HMAX > 8 ? 8 : HMAX;
+    constexpr int A = 32 / HT;
+    const size_t qrow = static_cast<size_t>(t.b) * a.H + static_cast<size_t>(t.g) * hpk;
+    over_atoms(c.k_atoms, abuf, region, [&](int c0, int n, const float* rows) {
+#pragma unroll 1
+      for (int h0 = 0; h0 < hpk; h0 += HT) {
+        float qreg[HT][E];
 #pragma unroll
-    for (int h = 0; h < HMAX; ++h)
+        for (int h = 0; h < HT; ++h)
 #pragma unroll
-      for (int e = 0; e < E; ++e) qreg[h][e] = h < hpk ? qs[h * D + lane * E + e] : 0.f;
-#pragma unroll 2
-    for (int a0 = warp * A; a0 < NA; a0 += NW * A) {
-      float v[32];
+          for (int e = 0; e < E; ++e) {
+            const size_t qi = (qrow + h0 + h) * D + lane * E + e;
+            qreg[h][e] = h0 + h >= hpk ? 0.f
+                         : c.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qi])
+                                    : static_cast<const float*>(a.q)[qi];
+          }
+        for (int a0 = warp * A; a0 < n; a0 += NW * A) {
+          float v[32];
 #pragma unroll
-      for (int i = 0; i < A; ++i) {
-        float kv[E];
-        const int at = a0 + i;
+          for (int i = 0; i < A; ++i) {
+            const int at = a0 + i;
+            float kv[E];
+            if (E == 4) {
+              const float4 k4 = at < n ? *reinterpret_cast<const float4*>(rows + at * D + lane * 4)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+              kv[0] = k4.x;
+              kv[1 % E] = k4.y;
+              kv[2 % E] = k4.z;
+              kv[3 % E] = k4.w;
+            } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e)
-          kv[e] = at < NA ? __ldg(c.k_atoms + static_cast<size_t>(at) * D + lane * E + e) : 0.f;
+              for (int e = 0; e < E; ++e) kv[e] = at < n ? rows[at * D + lane * E + e] : 0.f;
+            }
 #pragma unroll
-        for (int h = 0; h < HMAX; ++h) {
-          float d = 0.f;
+            for (int h = 0; h < HT; ++h) {
+              float d = 0.f;
 #pragma unroll
-          for (int e = 0; e < E; ++e) d = fmaf(qreg[h][e], kv[e], d);
-          v[i * HMAX + h] = d;
+              for (int e = 0; e < E; ++e) d = fmaf(qreg[h][e], kv[e], d);
+              v[i * HT + h] = d;
+            }
+          }
+#pragma unroll
+          for (int st = 0; st < 5; ++st) {
+            const int off = 16 >> st;
+            const bool upper = (lane & off) != 0;
+#pragma unroll
+            for (int i = 0; i < off; ++i) {
+              const float send = upper ? v[i] : v[i + off];
+              const float keep = upper ? v[i + off] : v[i];
+              v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            }
+          }
+          const int at = a0 + lane / HT, h = h0 + lane % HT;
+          if (at < n && h < hpk) qa[(c0 + at) * hpk + h] = v[0] * a.scale_log2;
         }
       }
-#pragma unroll
-      for (int st = 0; st < 5; ++st) {
-        const int off = 16 >> st;
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < off; ++i) {
-          const float send = upper ? v[i] : v[i + off];
-          const float keep = upper ? v[i + off] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-      }
-      const int at = a0 + lane / HMAX, h = lane % HMAX;
-      if (at < NA && h < hpk) qa[at * hpk + h] = v[0] * a.scale_log2;
-    }
+    });
   }
-  __syncthreads();
+  __syncthreads();                   // the table is complete; the logit store is free
 
-  // running maximum per head (identical in every thread), this thread's share
-  // of the partition, and the previous block's rescale and scale for the fold
-  float mrun[HMAX], lthr[HMAX], fprev[HMAX], inv_prev[HMAX];
+  // running maximum per head (identical in every thread) and this thread's
+  // share of the partition; the bounds of the last round stay in red2
+  // (double-buffered by round parity) for its fold.
+  float mrun[HMAX], lthr[HMAX];
 #pragma unroll
   for (int h = 0; h < HMAX; ++h) {
     mrun[h] = -INFINITY;
     lthr[h] = 0.f;
-    fprev[h] = 1.f;
-    inv_prev[h] = 0.f;
   }
+  auto fmax_op = [](float x, float y) { return fmaxf(x, y); };
+  auto fadd_op = [](float x, float y) { return x + y; };
   bool bad = false;
   const bool quad_heads = (hpk & 3) == 0;
 #pragma unroll 1
-  for (int blk = 0; blk < nblk; ++blk) {
-    const int kb = t.kbeg + blk * NT;
-    const int key = kb + tid;
-    const bool live = key < t.kend;
-    // this block's group has landed when at most slots - 2 later ones are pending
-    if (slots == 3)
-      ptx::cp_async_wait_group<1>();
-    else
-      ptx::cp_async_wait_group<0>();
-    uint32_t kw[MW], vw[MW];
-    const int slot = blk - (blk / slots) * slots;
-    load_row(cbuf + slot * 2 * W * NT, 0, kw);
-    load_row(cbuf + slot * 2 * W * NT, 1, vw);
-    if (!live)
+  for (int rd = 0; rd < nround && ok; ++rd) {
+    const int par = rd & 1;
+    const int kb = t.kbeg + rd * KR;
+    const int nk = round_keys(rd);
+    const int mine = rows_of(nk);
+    // ---- pass A: logits by table lookup into lg[key][h]; |V coefficient| sums
+    float tmax[HMAX];
 #pragma unroll
-      for (int w = 0; w < MW; ++w) kw[w] = vw[w] = 0u;
-    // the slot of the previous block, already read: own slots only, no barrier
-    stage_codes(blk + slots - 1);
-    // fold the previous block's integer weights into Wt (rescaled to the
-    // maximum they were taken against) and clear them
-    if (kb > t.kbeg)
+    for (int h = 0; h < HMAX; ++h) tmax[h] = -INFINITY;
+#pragma unroll 1
+    for (int i = 0; i < mine; ++i) {
+      wait_ring();
+      const int j = tid + i * NT;
+      uint32_t kw[MW];
+      ring_row(i, kw);
+      float s[HMAX];
 #pragma unroll
-      for (int h = 0; h < HMAX; ++h) {
-        if (h >= hpk) break;
-        for (int i = tid; i < NA; i += NT) {
-          const int j = h * NA + i;
-          Wt[j] = fmaf(Wt[j], fprev[h], static_cast<float>(static_cast<int32_t>(Wb[j])) * inv_prev[h]);
-          Wb[j] = 0u;
-        }
-      }
-    float sc[HMAX];
-#pragma unroll
-    for (int h = 0; h < HMAX; ++h) sc[h] = live ? 0.f : -INFINITY;
-    float csum = 0.f;                // sum of |V coefficient| of the key
-    if (live) {
+      for (int h = 0; h < HMAX; ++h) s[h] = 0.f;
 #pragma unroll
       for (int w = 0; w < MW; ++w) {
         const int idx = static_cast<int>(kw[w] >> 16);
-        const float cf = code_coeff(kw[w]);
-        if (cf == 0.f) continue;
-        if (idx >= NA) {
-          bad = true;
-          continue;
-        }
+        const bool in = idx < NA;
+        bad |= !in;
+        const float cf = in ? code_coeff(kw[w]) : 0.f;
         // an atom's logits of all heads sit side by side: 16-byte loads when
         // heads_per_kv is a multiple of 4
-        const float* row = qa + idx * hpk;
+        const float* row = qa + (in ? idx : 0) * hpk;
         if (quad_heads) {
 #pragma unroll
           for (int q4 = 0; q4 < HMAX / 4; ++q4)
             if (4 * q4 < hpk) {
               const float4 t4 = *reinterpret_cast<const float4*>(row + 4 * q4);
-              sc[4 * q4] = fmaf(cf, t4.x, sc[4 * q4]);
-              sc[4 * q4 + 1] = fmaf(cf, t4.y, sc[4 * q4 + 1]);
-              sc[4 * q4 + 2] = fmaf(cf, t4.z, sc[4 * q4 + 2]);
-              sc[4 * q4 + 3] = fmaf(cf, t4.w, sc[4 * q4 + 3]);
+              s[4 * q4] = fmaf(cf, t4.x, s[4 * q4]);
+              s[4 * q4 + 1] = fmaf(cf, t4.y, s[4 * q4 + 1]);
+              s[4 * q4 + 2] = fmaf(cf, t4.z, s[4 * q4 + 2]);
+              s[4 * q4 + 3] = fmaf(cf, t4.w, s[4 * q4 + 3]);
             }
         } else {
 #pragma unroll
           for (int h = 0; h < HMAX; ++h)
-            if (h < hpk) sc[h] = fmaf(cf, row[h], sc[h]);
+            if (h < hpk) s[h] = fmaf(cf, row[h], s[h]);
         }
       }
-      const float bb = bias2(a, t, key);
+      if (VST) {
+        uint32_t vw[MW];
+        read_row(vst + (quads ? j * 4 : j), KR, vw);
+        float csum = 0.f;
 #pragma unroll
-      for (int h = 0; h < HMAX; ++h) sc[h] += bb;
-#pragma unroll
-      for (int w = 0; w < MW; ++w) csum += fabsf(code_coeff(vw[w]));
-    }
-    // block maxima per head
-#pragma unroll
-    for (int h = 0; h < HMAX; ++h) {
-      if (h >= hpk) break;
-      float v = sc[h];
-      for (int x = 16; x >= 1; x >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, x));
-      if (lane == 0) red[warp][h] = v;
-    }
-    __syncthreads();                 // red complete; Wb folded and clear
-    float p[HMAX];
-#pragma unroll
-    for (int h = 0; h < HMAX; ++h) {
-      if (h >= hpk) {
-        p[h] = 0.f;
-        continue;
+        for (int w = 0; w < MW; ++w) csum += fabsf(code_coeff(vw[w]));
+        cs[j] = csum;
       }
-      float bm = -INFINITY;
+      const float bb = bias2(a, t, kb + j);
+      float* dst = lg + j * hpk;
+      if (quad_heads) {
 #pragma unroll
-      for (int w = 0; w < NW; ++w) bm = fmaxf(bm, red[w][h]);
-      const float mn = fmaxf(mrun[h], bm);
-      const float f = (mn == -INFINITY) ? 1.f : exp2f(mrun[h] - mn);
-      mrun[h] = mn;
-      fprev[h] = f;
-      p[h] = exp2f(sc[h] - (mn == -INFINITY ? 0.f : mn));
-      lthr[h] = fmaf(lthr[h], f, p[h]);
+        for (int q4 = 0; q4 < HMAX / 4; ++q4)
+          if (4 * q4 < hpk)
+            *reinterpret_cast<float4*>(dst + 4 * q4) =
+                make_float4(s[4 * q4] + bb, s[4 * q4 + 1] + bb, s[4 * q4 + 2] + bb, s[4 * q4 + 3] + bb);
+      } else {
+#pragma unroll
+        for (int h = 0; h < HMAX; ++h)
+          if (h < hpk) dst[h] = s[h] + bb;
+      }
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h) tmax[h] = fmaxf(tmax[h], s[h] + bb);
+      issue_row(kbase, kb, mine, i + P);   // the slot's row has been used: refill it
     }
-    // per head: bound on the block's weight sums, summed in a fixed order
+    if (!VST) prime(vbase, kb, mine);  // pass B's V rows come in across the barrier
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
       if (h >= hpk) break;
-      float v = p[h] * csum;
-      for (int x = 16; x >= 1; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
-      if (lane == 0) red2[warp][h] = v;
+      float v = tmax[h];
+#pragma unroll
+      for (int x = 16; x >= 1; x >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, x));
+      if (lane == 0) red[h][warp] = v;
     }
-    __syncthreads();                 // red2 complete
-    float scale[HMAX];
+    __syncthreads();                 // red complete; the last round's atomics done
+    // ---- pass B: new maximum; fold of the last round's Wb into Wt; weights
+    // p into lg; partition; bound on any atom's weight sum
+    float mn[HMAX];
+    cta_reduce_heads<HMAX, NW>(red, hpk, lane, -INFINITY, mn, fmax_op);
+    {
+      float unit[HMAX];
+      if (rd > 0) cta_reduce_heads<HMAX, NW>(red2[par ^ 1], hpk, lane, 0.f, unit, fadd_op);
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h) {
+        if (h >= hpk) break;
+        mn[h] = fmaxf(mrun[h], mn[h]);
+        const float f = (mn[h] == -INFINITY) ? 1.f : exp2f(mrun[h] - mn[h]);
+        mrun[h] = mn[h];
+        lthr[h] *= f;
+        if (rd > 0) {
+          // Wt and the last round's Wb are both relative to the previous
+          // maximum: add them and rescale to the new one; clear Wb
+          const float sc = block_weight_scale(unit[h]);
+          const float u = sc > 0.f ? 1.f / sc : 0.f;
+          for (int i = h * NA + tid; i < (h + 1) * NA; i += NT) {
+            Wt[i] = (Wt[i] + static_cast<float>(static_cast<int32_t>(Wb[i])) * u) * f;
+            Wb[i] = 0u;
+          }
+        }
+        if (mn[h] == -INFINITY) mn[h] = 0.f;          // all masked so far: weights 0
+      }
+    }
+    float bnd[HMAX];
+#pragma unroll
+    for (int h = 0; h < HMAX; ++h) bnd[h] = 0.f;
+#pragma unroll 2
+    for (int i = 0; i < mine; ++i) {
+      const int j = tid + i * NT;
+      float csum;
+      if (VST) {
+        csum = cs[j];
+      } else {
+        wait_ring();
+        uint32_t vw[MW];
+        ring_row(i, vw);
+        csum = 0.f;
+#pragma unroll
+        for (int w = 0; w < MW; ++w) csum += fabsf(code_coeff(vw[w]));
+        issue_row(vbase, kb, mine, i + P);
+      }
+      float* src = lg + j * hpk;
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h)
+        if (h < hpk) {
+          const float p = exp2f(src[h] - mn[h]);
+          src[h] = p;
+          lthr[h] += p;
+          bnd[h] = fmaf(p, csum, bnd[h]);
+        }
+    }
+    if (!VST) prime(vbase, kb, mine);  // pass C's V rows come in across the barrier
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
-      float bound = 0.f;
-      if (h < hpk)
+      if (h >= hpk) break;
+      float v = bnd[h];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) bound += red2[w][h];
-      scale[h] = block_weight_scale(bound);
-      inv_prev[h] = scale[h] > 0.f ? 1.f / scale[h] : 0.f;
+      for (int x = 16; x >= 1; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
+      if (lane == 0) red2[par][h][warp] = v;
     }
-    float ps[HMAX];                  // weights already in fixed-point units
+    __syncthreads();                 // red2 complete; Wb folded and clear
+    // ---- pass C: the weights into Wb, in fixed point
+    float scale[HMAX];
+    cta_reduce_heads<HMAX, NW>(red2[par], hpk, lane, 0.f, scale, fadd_op);
 #pragma unroll
-    for (int h = 0; h < HMAX; ++h) ps[h] = p[h] * scale[h];
-    if (live) {
+    for (int h = 0; h < HMAX; ++h) scale[h] = h < hpk ? block_weight_scale(scale[h]) : 0.f;
+#pragma unroll 1
+    for (int i = 0; i < mine; ++i) {
+      const int j = tid + i * NT;
+      uint32_t vw[MW];
+      if (VST) {
+        read_row(vst + (quads ? j * 4 : j), KR, vw);
+      } else {
+        wait_ring();
+        ring_row(i, vw);
+      }
+      float ps[HMAX];                // weights in fixed-point units
+      const float* src = lg + j * hpk;
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h) ps[h] = h < hpk ? src[h] * scale[h] : 0.f;
 #pragma unroll
       for (int w = 0; w < MW; ++w) {
         const int idx = static_cast<int>(vw[w] >> 16);
         const float cf = code_coeff(vw[w]);
-        if (cf == 0.f) continue;
-        if (idx >= NA) {
-          bad = true;
-          continue;
-        }
+        const bool in = idx < NA;
+        bad |= !in;
+        if (!in || cf == 0.f) continue;
+        uint32_t* wrow = Wb + idx;
 #pragma unroll
         for (int h = 0; h < HMAX; ++h)
-          if (h < hpk && p[h] != 0.f)
-            atomicAdd(Wb + h * NA + idx, static_cast<uint32_t>(__float2int_rn(ps[h] * cf)));
+          if (h < hpk && ps[h] != 0.f)
+            atomicAdd(wrow + h * NA, static_cast<uint32_t>(__float2int_rn(ps[h] * cf)));
       }
+      if (!VST) issue_row(vbase, kb, mine, i + P);
     }
-    __syncthreads();                 // Wb complete before the next fold; red, red2 free
+    // this thread is done with its rows of the round: the next round's copies
+    // start now, across the barrier
+    if (rd + 1 < nround) start_round(rd + 1);
   }
-  // the last block's weights
+  ptx::cp_async_wait_group<0>();     // no copy left in flight
+  __syncthreads();                   // the last round's atomics done
+  // the last round's weights
+  if (nround > 0 && ok) {
+    float unit[HMAX];
+    cta_reduce_heads<HMAX, NW>(red2[(nround - 1) & 1], hpk, lane, 0.f, unit, fadd_op);
 #pragma unroll
-  for (int h = 0; h < HMAX; ++h) {
-    if (h >= hpk) break;
-    for (int i = tid; i < NA; i += NT) {
-      const int j = h * NA + i;
-      Wt[j] = fmaf(Wt[j], fprev[h], static_cast<float>(static_cast<int32_t>(Wb[j])) * inv_prev[h]);
+    for (int h = 0; h < HMAX; ++h) {
+      if (h >= hpk) break;
+      const float sc = block_weight_scale(unit[h]);
+      const float u = sc > 0.f ? 1.f / sc : 0.f;
+      for (int i = h * NA + tid; i < (h + 1) * NA; i += NT)
+        Wt[i] += static_cast<float>(static_cast<int32_t>(Wb[i])) * u;
     }
   }
   // the partition: every thread's share, summed in a fixed order
@@ -382,67 +608,134 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   for (int h = 0; h < HMAX; ++h) {
     if (h >= hpk) break;
     float v = lthr[h];
+#pragma unroll
     for (int x = 16; x >= 1; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
-    if (lane == 0) red[warp][h] = v;
+    if (lane == 0) red[h][warp] = v;
   }
   __syncthreads();
+  {
+    float L[HMAX];
+    cta_reduce_heads<HMAX, NW>(red, hpk, lane, 0.f, L, fadd_op);
+#pragma unroll
+    for (int h = 0; h < HMAX; ++h)
+      if (h < hpk && tid == h) {
+        hM[h] = mrun[h];
+        hL[h] = L[h];
+      }
+  }
+  // (hM, hL are read after the barriers of the atom copies below)
   if (bad) atomicOr(a.err, kErrBadCodes);
   if (threadIdx.x == 0) ptx::grid_launch_dependents();
 
-  // acc[h][d] = sum over atoms of Wt[h][atom] * vatom[atom][d]: warp w takes
-  // atoms w, w+8, ... with lanes across D, then the warps add into accb
-  {
-    float acc[HMAX][E];
-#pragma unroll
-    for (int h = 0; h < HMAX; ++h)
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
-#pragma unroll 16
-    for (int at = warp; at < NA; at += NW) {
-      float vv[E];
-#pragma unroll
-      for (int e = 0; e < E; ++e) vv[e] = __ldg(c.v_atoms + static_cast<size_t>(at) * D + lane * E + e);
-#pragma unroll
-      for (int h = 0; h < HMAX; ++h) {
-        if (h >= hpk) break;
-        const float wgt = Wt[h * NA + at];
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[h][e] = fmaf(wgt, vv[e], acc[h][e]);
+  // acc[h][d] = sum over atoms of Wt[h][atom] * vatom[atom][d]: the V atoms
+  // come through the round region (and the ring) in chunks. Thread tid owns
+  // column quad qd = tid % Q of head h = (tid / Q) % HMAX for atom share ag =
+  // tid / (Q * HMAX) (atoms ag, ag + AG, ...), summing its atoms in order; the
+  // AG shares then add in order.
+  constexpr int Q = D / 4;
+  constexpr int AG = NT / (Q * HMAX);                  // atom shares: 1 .. 8
+  static_assert(AG >= 1 && Q * HMAX * AG == NT, "threads cover quads x heads x shares");
+  const int qd = tid % Q, hh = (tid / Q) % HMAX, ag = tid / (Q * HMAX);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (ok)
+    over_atoms(c.v_atoms, reinterpret_cast<float*>(ring), P * W * NT + KR * coded_key_words(W, hpk),
+               [&](int c0, int n, const float* rows) {
+                 if (hh < hpk) {
+                   const float* wr = Wt + hh * NA + c0;
+#pragma unroll 4
+                   for (int at = ag; at < n; at += AG) {
+                     const float4 vv = *reinterpret_cast<const float4*>(rows + at * D + qd * 4);
+                     const float wgt = wr[at];
+                     acc.x = fmaf(wgt, vv.x, acc.x);
+                     acc.y = fmaf(wgt, vv.y, acc.y);
+                     acc.z = fmaf(wgt, vv.z, acc.z);
+                     acc.w = fmaf(wgt, vv.w, acc.w);
+                   }
+                 }
+               });
+  if (!ok) return;                   // a copy never landed (flagged): no state out
+  __syncthreads();                   // the atom buffers are free
+  if (AG > 1) {
+    float4* sh = reinterpret_cast<float4*>(ring);      // [AG][HMAX][Q] (the region holds >= 8 KB)
+    sh[(ag * HMAX + hh) * Q + qd] = acc;
+    __syncthreads();
+    if (ag == 0)
+      for (int g2 = 1; g2 < AG; ++g2) {
+        const float4 o = sh[(g2 * HMAX + hh) * Q + qd];
+        acc.x += o.x;
+        acc.y += o.y;
+        acc.z += o.z;
+        acc.w += o.w;
       }
-    }
-    // the warps' sums in warp order (deterministic), through accb
-    for (int w = 0; w < NW; ++w) {
-      if (warp == w) {
+  }
+  const bool owner = ag == 0 && hh < hpk;
+
+  // The state goes out as store_partial writes a single slot (m in natural-log units).
+  if (owner) *reinterpret_cast<float4*>(a.part_acc + state_index(a, t, hh) * D + qd * 4) = acc;
+  if (tid < hpk) {
+    const size_t si = state_index(a, t, tid);
+    a.part_m[si] = (hL[tid] == 0.f) ? -INFINITY : hM[tid] * kLn2;
+    a.part_l[si] = hL[tid];
+  }
+  if (!a.merge) return;
+  if (t.kbeg == 0 && t.kend == t.n) {
+    // The tile is the whole sequence: fold the carry (USearch linear algebra,
+    // DenseAttendConfig::carry) and write out / state_out from here.
+    const size_t row0 = static_cast<size_t>(t.b) * a.H + static_cast<size_t>(t.g) * hpk;
+    if (owner) {
+      const size_t r = row0 + hh;
+      const float Lh = hL[hh];
+      float Mh = Lh == 0.f ? -INFINITY : hM[hh] * kLn2;
+      const bool has_carry = a.cl != nullptr && a.cl[r] != 0.f;
+      float wt = Lh == 0.f ? 0.f : 1.f, wc = 0.f;
+      if (has_carry) {
+        const float cmr = a.cm[r];
+        const float M = fmaxf(Mh, cmr);
+        wt = Lh == 0.f ? 0.f : expf(Mh - M);
+        wc = expf(cmr - M);
+        Mh = M;
+      }
+      const float Lt = fmaf(Lh, wt, has_carry ? a.cl[r] * wc : 0.f);
+      float y[4] = {acc.x * wt, acc.y * wt, acc.z * wt, acc.w * wt};
+      if (has_carry) {
+        const float4 cv = *reinterpret_cast<const float4*>(a.cacc + r * D + qd * 4);
+        y[0] = fmaf(cv.x, wc, y[0]);
+        y[1] = fmaf(cv.y, wc, y[1]);
+        y[2] = fmaf(cv.z, wc, y[2]);
+        y[3] = fmaf(cv.w, wc, y[3]);
+      }
+      if (a.oacc) *reinterpret_cast<float4*>(a.oacc + r * D + qd * 4) = make_float4(y[0], y[1], y[2], y[3]);
+      if (a.out) {
+        float o[4];
 #pragma unroll
-        for (int h = 0; h < HMAX; ++h) {
-          if (h >= hpk) break;
-#pragma unroll
-          for (int e = 0; e < E; ++e) accb[h * D + lane * E + e] += acc[h][e];
+        for (int e = 0; e < 4; ++e) o[e] = Lt == 0.f ? 0.f : __fdiv_rn(y[e], Lt);
+        if (a.out_bf16) {
+          __nv_bfloat162* dst =
+              reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.out) + r * D + qd * 4);
+          dst[0] = __floats2bfloat162_rn(o[0], o[1]);
+          dst[1] = __floats2bfloat162_rn(o[2], o[3]);
+        } else {
+          *reinterpret_cast<float4*>(static_cast<float*>(a.out) + r * D + qd * 4) =
+              make_float4(o[0], o[1], o[2], o[3]);
         }
       }
-      __syncthreads();
+      if (qd == 0) {
+        smM[hh] = Lt == 0.f ? -INFINITY : Mh;
+        smL[hh] = Lt;
+      }
     }
-  }
-  // the state goes out exactly as store_partial writes a single slot
-  for (int i = tid; i < hpk * D; i += NT) {
-    const int h = i / D, d = i % D;
-    a.part_acc[state_index(a, t, h) * D + d] = accb[i];
-  }
-#pragma unroll
-  for (int h = 0; h < HMAX; ++h)
-    if (h < hpk && tid == h) {
-      float L = 0.f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) L += red[w][h];
-      const size_t si = state_index(a, t, h);
-      a.part_m[si] = (L == 0.f) ? -INFINITY : mrun[h] * kLn2;
-      a.part_l[si] = L;
-    }
-  if (a.merge) {
+    // m and l of the state out are written after every thread has read the
+    // carry (state out may alias it)
     __syncthreads();
-    if (tid < 128)
-      finish_segment<D, HMAX>(a, t, tid, smM, smL, smC, &smFlag, qa, hpk * NA, 0u, NamedSync128{});
+    if (a.om && tid < hpk) {
+      a.om[row0 + tid] = smM[tid];
+      a.ol[row0 + tid] = smL[tid];
+    }
+    return;
   }
+  __syncthreads();
+  if (tid < 128)
+    finish_segment<D, HMAX>(a, t, tid, smM, smL, smC, &smFlag, qa, hpk * NA, 0u, NamedSync128{});
 }
 
 }  // namespace gqa

@@ -61,9 +61,15 @@ cudaError_t prepare_f32(int* resident) {
                                                        C::kThreads, C::kSmemBytes);
 }
 
-// the coded kernel's largest dynamic shared memory: 16 code words, the largest tables
-constexpr int kCodedMaxSmem = static_cast<int>(gqa::coded_smem_bytes(gqa::kMaxCodeWords, 1,
-                                                                      gqa::kCodedMaxTableEntries));
+// the coded kernel's dynamic shared memory: every call's plan fits its budget,
+// which leaves room under the 227 KB of a CTA for the kernel's static shared
+// memory (3.4 KB at most); the largest tables still leave a ring row and the
+// smallest round store
+constexpr int kCodedMaxSmem = gqa::kCodedSmemBudget;
+static_assert(kCodedMaxSmem + 4096 <= 227 * 1024, "coded shared memory under the per-CTA limit");
+static_assert(gqa::coded_ring_fits(1, gqa::kMaxCodeWords, 1, gqa::kCodedMaxTableEntries) &&
+                  gqa::coded_ring_fits(1, gqa::kMaxCodeWords, 16, gqa::kCodedMaxTableEntries / 16),
+              "the largest coded tables fit beside a ring row and the smallest round store");
 
 template <int D, int HMAX, int MW>
 cudaError_t prepare_coded() {
@@ -291,7 +297,7 @@ gqa_status plan_impl(int32_t batch, int32_t G, int32_t max_seq_len, int64_t tota
 }
 
 // Host-side validation and planning shared by workspace_size and attend.
-gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
+gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device, int per_sm_override = 0) {
   if (!p || p->struct_size != sizeof(gqa_decode_params)) return GQA_ERR_INVALID_ARGUMENT;
   r->B = p->batch;
   r->H = p->num_heads;
@@ -349,6 +355,7 @@ gqa_status resolve(const gqa_decode_params* p, Resolved* r, bool need_device) {
     r->sm_count = di->sm_count;
     r->per_sm = per_sm > 0 ? per_sm : 1;
   }
+  if (per_sm_override > 0) r->per_sm = per_sm_override;
   // split plan
   if (p->num_splits > 0) {
     r->S = p->num_splits;
@@ -448,6 +455,7 @@ cudaError_t launch_coded(Launch& l, int hp, int mw, const PartitionArgs& a, cons
   if (hp == 8) return launch_coded_hp<D, 8>(l, mw, a, c);
   return launch_coded_hp<D, 16>(l, mw, a, c);
 }
+
 
 cudaError_t launch_partition(const Resolved& r, const PartitionArgs& a, const CUtensorMap* tk,
                              const CUtensorMap* tv, cudaStream_t st, bool early) {
@@ -634,24 +642,52 @@ gqa_status gqa_decode_append_attend(const gqa_decode_params* p, const void* k_ne
                      k_new, v_new);
 }
 
-gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_codes* codes,
-                                   gqa_stream_t stream) {
+// Validation and the split plan of a coded call: everything as gqa_decode_attend
+// would check it, with the code arrays standing in for the caches (their dtype
+// is the queries'), and the plan made for the coded kernel's occupancy (one
+// CTA of 512 threads per SM).
+static gqa_status resolve_coded(const gqa_decode_params* p, const gqa_kv_codes* codes, gqa_decode_params* pc,
+                                Resolved* r) {
   if (!p || !codes || p->struct_size != sizeof(gqa_decode_params)) return GQA_ERR_INVALID_ARGUMENT;
   if (codes->words < 1 || codes->words > 16 || codes->n_atoms < 1 || codes->n_atoms > 65536)
     return GQA_ERR_INVALID_ARGUMENT;
-  // Validate everything else as gqa_decode_attend would, with the code arrays
-  // standing in for the caches (their dtype is the queries').
-  gqa_decode_params pc = *p;
-  pc.k = codes->k_codes;
-  pc.v = codes->v_codes;
-  pc.kv_dtype = p->q_dtype;
-  Resolved r;
-  gqa_status st = resolve(&pc, &r, true);
+  *pc = *p;
+  pc->k = codes->k_codes;
+  pc->v = codes->v_codes;
+  pc->kv_dtype = p->q_dtype;
+  gqa_status st = resolve(pc, r, true, 1);
   if (st != GQA_OK) return st;
-  if (r.B > 0 && r.max_len > 0 && (!codes->k_atoms || !codes->v_atoms)) return GQA_ERR_INVALID_ARGUMENT;
+  if (r->B > 0 && r->max_len > 0 && (!codes->k_atoms || !codes->v_atoms)) return GQA_ERR_INVALID_ARGUMENT;
   if ((reinterpret_cast<uintptr_t>(codes->k_atoms) | reinterpret_cast<uintptr_t>(codes->v_atoms)) & 15u)
     return GQA_ERR_SHAPE_MISMATCH;
-  if (static_cast<int64_t>(r.hpk) * codes->n_atoms > gqa::kCodedMaxTableEntries) return GQA_ERR_INVALID_ARGUMENT;
+  // rows of 4k words are read 16 bytes at a time
+  if ((codes->words & 3) == 0 &&
+      ((reinterpret_cast<uintptr_t>(codes->k_codes) | reinterpret_cast<uintptr_t>(codes->v_codes)) & 15u))
+    return GQA_ERR_SHAPE_MISMATCH;
+  if (static_cast<int64_t>(r->hpk) * codes->n_atoms > gqa::kCodedMaxTableEntries ||
+      !gqa::coded_ring_fits(1, codes->words, r->hpk, codes->n_atoms))
+    return GQA_ERR_INVALID_ARGUMENT;
+  return GQA_OK;
+}
+
+gqa_status gqa_decode_coded_workspace_size(const gqa_decode_params* p, const gqa_kv_codes* codes, size_t* bytes,
+                                           int32_t* num_splits, int32_t* chunk_len) {
+  gqa_decode_params pc;
+  Resolved r;
+  gqa_status st = resolve_coded(p, codes, &pc, &r);
+  if (st != GQA_OK) return st;
+  if (bytes) *bytes = r.bytes;
+  if (num_splits) *num_splits = r.S;
+  if (chunk_len) *chunk_len = r.chunk;
+  return GQA_OK;
+}
+
+gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_codes* codes,
+                                   gqa_stream_t stream) {
+  gqa_decode_params pc;
+  Resolved r;
+  gqa_status st = resolve_coded(p, codes, &pc, &r);
+  if (st != GQA_OK) return st;
   const size_t smem = gqa::coded_smem_bytes(codes->words, r.hpk, codes->n_atoms);
   if (!p->workspace || p->workspace_bytes < r.bytes) return GQA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(p->workspace) & 255u) return GQA_ERR_WORKSPACE;
@@ -675,7 +711,7 @@ gqa_status gqa_decode_attend_coded(const gqa_decode_params* p, const gqa_kv_code
     return GQA_ERR_DEVICE;
   }
   const unsigned grid = static_cast<unsigned>(r.B) * r.S * r.G;
-  Launch l(grid, 256, smem, cs, (p->flags & GQA_FLAG_EARLY_START) != 0);
+  Launch l(grid, gqa::kCodedThreads, smem, cs, (p->flags & GQA_FLAG_EARLY_START) != 0);
   cudaError_t e;
   const int hp = r.hpk <= 4 ? 4 : (r.hpk <= 8 ? 8 : 16);
   const int mw = codes->words <= 4 ? 4 : (codes->words <= 8 ? 8 : 16);

@@ -259,93 +259,103 @@ __device__ __forceinline__ void merge_segment(const PartitionArgs& a, const Tile
   sync();
 
   const int qd = tid / GC, cg = tid % GC;
-  float4 acc[HP];
-#pragma unroll
-  for (int h = 0; h < HP; ++h) acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (staged) {
-    // Issue every load of a batch of U splits x HP rows before any arithmetic:
-    // the loads are independent, so the batch costs one trip to L2.
-    constexpr int U = HP <= 8 ? 2 : 1;
+  // heads in groups of HB (at most 8 float4 accumulators per thread)
+  constexpr int HB = HP > 8 ? 8 : HP;
 #pragma unroll 1
-    for (int c0 = cg; c0 < nsplit; c0 += U * GC) {
-      float4 v[U][HP];
-      float w[U][HP];
+  for (int h0 = 0; h0 < hpk; h0 += HB) {
+    float4 acc[HB];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c = c0 + u * GC;
+    for (int hh = 0; hh < HB; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (staged) {
+      // Issue every load of a batch of U splits x HB rows before any arithmetic:
+      // the loads are independent, so the batch costs one trip to L2.
+      constexpr int U = HB <= 4 ? 2 : 1;
+#pragma unroll 1
+      for (int c0 = cg; c0 < nsplit; c0 += U * GC) {
+        float4 v[U][HB];
+        float w[U][HB];
 #pragma unroll
-        for (int h = 0; h < HP; ++h) {
-          const bool live = h < hpk && c < nsplit;
-          w[u][h] = live ? wm[h * nsplit + c] : 0.f;
-          v[u][h] = live ? __ldcg(reinterpret_cast<const float4*>(a.part_acc + ((row0 + h) * S + c) * D) + qd)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < U; ++u) {
+          const int c = c0 + u * GC;
+#pragma unroll
+          for (int hh = 0; hh < HB; ++hh) {
+            const int h = h0 + hh;
+            const bool live = h < hpk && c < nsplit;
+            w[u][hh] = live ? wm[h * nsplit + c] : 0.f;
+            v[u][hh] = live ? __ldcg(reinterpret_cast<const float4*>(a.part_acc + ((row0 + h) * S + c) * D) + qd)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int hh = 0; hh < HB; ++hh) {
+            acc[hh].x = fmaf(v[u][hh].x, w[u][hh], acc[hh].x);
+            acc[hh].y = fmaf(v[u][hh].y, w[u][hh], acc[hh].y);
+            acc[hh].z = fmaf(v[u][hh].z, w[u][hh], acc[hh].z);
+            acc[hh].w = fmaf(v[u][hh].w, w[u][hh], acc[hh].w);
+          }
+      }
+    } else {
+      // Too many splits to stage their weights: recompute them (slower).
+      for (int c = cg; c < nsplit; c += GC) {
+#pragma unroll
+        for (int hh = 0; hh < HB; ++hh) {
+          const int h = h0 + hh;
+          if (h >= hpk) break;
+          const size_t si = (row0 + h) * S + c;
+          const float lc = __ldcg(a.part_l + si);
+          const float w = (lc != 0.f && smM[h] != -INFINITY) ? expf(__ldcg(a.part_m + si) - smM[h]) : 0.f;
+          if (w == 0.f) continue;
+          const float4 vv = __ldcg(reinterpret_cast<const float4*>(a.part_acc + si * D) + qd);
+          acc[hh].x = fmaf(vv.x, w, acc[hh].x);
+          acc[hh].y = fmaf(vv.y, w, acc[hh].y);
+          acc[hh].z = fmaf(vv.z, w, acc[hh].z);
+          acc[hh].w = fmaf(vv.w, w, acc[hh].w);
         }
       }
+    }
 #pragma unroll
-      for (int u = 0; u < U; ++u)
+    for (int hh = 0; hh < HB; ++hh) {
+      if (h0 + hh >= hpk) break;
 #pragma unroll
-        for (int h = 0; h < HP; ++h) {
-          acc[h].x = fmaf(v[u][h].x, w[u][h], acc[h].x);
-          acc[h].y = fmaf(v[u][h].y, w[u][h], acc[h].y);
-          acc[h].z = fmaf(v[u][h].z, w[u][h], acc[h].z);
-          acc[h].w = fmaf(v[u][h].w, w[u][h], acc[h].w);
+      for (int x = 1; x < GC; x <<= 1) {
+        acc[hh].x += __shfl_xor_sync(0xffffffffu, acc[hh].x, x);
+        acc[hh].y += __shfl_xor_sync(0xffffffffu, acc[hh].y, x);
+        acc[hh].z += __shfl_xor_sync(0xffffffffu, acc[hh].z, x);
+        acc[hh].w += __shfl_xor_sync(0xffffffffu, acc[hh].w, x);
+      }
+    }
+    if (cg == 0) {
+#pragma unroll
+      for (int hh = 0; hh < HB; ++hh) {
+        const int h = h0 + hh;
+        if (h >= hpk) break;
+        const size_t r = row0 + h;
+        const float wc = smC[h];
+        float y[4] = {acc[hh].x, acc[hh].y, acc[hh].z, acc[hh].w};
+        if (wc != 0.f) {
+          const float4 cv = *reinterpret_cast<const float4*>(a.cacc + r * D + qd * 4);
+          y[0] = fmaf(cv.x, wc, y[0]);
+          y[1] = fmaf(cv.y, wc, y[1]);
+          y[2] = fmaf(cv.z, wc, y[2]);
+          y[3] = fmaf(cv.w, wc, y[3]);
         }
-    }
-  } else {
-    // Too many splits to stage their weights: recompute them (slower).
-    for (int c = cg; c < nsplit; c += GC) {
-      for (int h = 0; h < hpk && h < HP; ++h) {
-        const size_t si = (row0 + h) * S + c;
-        const float lc = __ldcg(a.part_l + si);
-        const float w = (lc != 0.f && smM[h] != -INFINITY) ? expf(__ldcg(a.part_m + si) - smM[h]) : 0.f;
-        if (w == 0.f) continue;
-        const float4 vv = __ldcg(reinterpret_cast<const float4*>(a.part_acc + si * D) + qd);
-        acc[h].x = fmaf(vv.x, w, acc[h].x);
-        acc[h].y = fmaf(vv.y, w, acc[h].y);
-        acc[h].z = fmaf(vv.z, w, acc[h].z);
-        acc[h].w = fmaf(vv.w, w, acc[h].w);
-      }
-    }
-  }
+        if (a.oacc) *reinterpret_cast<float4*>(a.oacc + r * D + qd * 4) = make_float4(y[0], y[1], y[2], y[3]);
+        if (a.out) {
+          const float L = smL[h];
+          float o[4];
 #pragma unroll
-  for (int h = 0; h < HP; ++h) {
-    if (h >= hpk) break;
-#pragma unroll
-    for (int x = 1; x < GC; x <<= 1) {
-      acc[h].x += __shfl_xor_sync(0xffffffffu, acc[h].x, x);
-      acc[h].y += __shfl_xor_sync(0xffffffffu, acc[h].y, x);
-      acc[h].z += __shfl_xor_sync(0xffffffffu, acc[h].z, x);
-      acc[h].w += __shfl_xor_sync(0xffffffffu, acc[h].w, x);
-    }
-  }
-  if (cg == 0) {
-#pragma unroll
-    for (int h = 0; h < HP; ++h) {
-      if (h >= hpk) break;
-      const size_t r = row0 + h;
-      const float wc = smC[h];
-      float y[4] = {acc[h].x, acc[h].y, acc[h].z, acc[h].w};
-      if (wc != 0.f) {
-        const float4 cv = *reinterpret_cast<const float4*>(a.cacc + r * D + qd * 4);
-        y[0] = fmaf(cv.x, wc, y[0]);
-        y[1] = fmaf(cv.y, wc, y[1]);
-        y[2] = fmaf(cv.z, wc, y[2]);
-        y[3] = fmaf(cv.w, wc, y[3]);
-      }
-      if (a.oacc) *reinterpret_cast<float4*>(a.oacc + r * D + qd * 4) = make_float4(y[0], y[1], y[2], y[3]);
-      if (a.out) {
-        const float L = smL[h];
-        float o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = (L == 0.f) ? 0.f : __fdiv_rn(y[e], L);
-        if (a.out_bf16) {
-          __nv_bfloat162* dst =
-              reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.out) + r * D + qd * 4);
-          dst[0] = __floats2bfloat162_rn(o[0], o[1]);
-          dst[1] = __floats2bfloat162_rn(o[2], o[3]);
-        } else {
-          *reinterpret_cast<float4*>(static_cast<float*>(a.out) + r * D + qd * 4) =
-              make_float4(o[0], o[1], o[2], o[3]);
+          for (int e = 0; e < 4; ++e) o[e] = (L == 0.f) ? 0.f : __fdiv_rn(y[e], L);
+          if (a.out_bf16) {
+            __nv_bfloat162* dst =
+                reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.out) + r * D + qd * 4);
+            dst[0] = __floats2bfloat162_rn(o[0], o[1]);
+            dst[1] = __floats2bfloat162_rn(o[2], o[3]);
+          } else {
+            *reinterpret_cast<float4*>(static_cast<float*>(a.out) + r * D + qd * 4) =
+                make_float4(o[0], o[1], o[2], o[3]);
+          }
         }
       }
     }

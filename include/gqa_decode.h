@@ -237,11 +237,19 @@ typedef struct {
  * are ignored; q is fp32 or bf16; everything else (offsets, carry, bias,
  * partials, outputs, workspace, flags) as gqa_decode_attend. A code word naming
  * an atom >= n_atoms is skipped and flags GQA_ERR_BAD_CODES in the device error
- * word. The per-atom value weights are summed per block of 256 keys in 32-bit
- * fixed point, scaled to the block's largest possible sum (rounding error at
- * most 2^-31 of it per weight), so results are bit-reproducible. */
+ * word. The per-atom value weights are summed per super-block of 512 or 1024
+ * keys in 32-bit fixed point, scaled to the super-block's largest possible sum
+ * (rounding error at most 2^-31 of it per weight), so results are
+ * bit-reproducible. The split plan is the coded kernel's own (one CTA of 512
+ * threads per SM), so size the workspace with gqa_decode_coded_workspace_size. */
 gqa_status gqa_decode_attend_coded(const gqa_decode_params* params, const gqa_kv_codes* codes,
                                    gqa_stream_t stream);
+
+/* Workspace bytes and split plan of gqa_decode_attend_coded for these params
+ * and codes (any output pointer may be NULL). Host only; reads the current
+ * device's SM count. Validates as gqa_decode_attend_coded does. */
+gqa_status gqa_decode_coded_workspace_size(const gqa_decode_params* params, const gqa_kv_codes* codes,
+                                           size_t* bytes, int32_t* num_splits, int32_t* chunk_len);
 
 /* Index-selected attention as an additive bias (metrale glm5next_dsa_ref,
  * `topk_to_mask`: the attention reads a mask built from an index row; repeated
