@@ -239,9 +239,16 @@ int nt_of(int hpk) { return hpk <= 8 ? 1 : 2; }
 // the CTAs fill the `resident` slots. A last partial wave costs as much as
 // max(its CTAs, sm_count) CTAs would (each CTA's own stream is bounded). The
 // plan minimises
-//     waves * (chunk_len + 128) + 4 * num_splits
+//     waves * (chunk_len + 128) + 4 * num_splits + merge
 // (128 rows ~ a CTA's fixed prologue/epilogue, 4 rows ~ one more partial state
-// in the merge), ties going to fewer splits.
+// in the merge), ties going to fewer splits. merge = 256 rows when the
+// sequences are long (>= 2048 keys) and there is more than one split: the
+// segment's last CTA takes its ticket and pulls the other splits' states from
+// L2 after its own stream, about 3-4 us on B200, which only counts against
+// long streams (short ones are bound by each CTA's latency, and splitting
+// them pays). Measured on B200, 16 sequences x 8 KV heads x 4096 keys: 1
+// split (128 CTAs) streams as fast as 2 back to back and ends a lone call
+// ~4 us sooner.
 // Ragged batch (total_rows below batch * max_seq_len): the tiles are uneven, so
 // the plan aims at ~8 waves of CTAs and lets the block scheduler balance them.
 gqa_status plan_impl(int32_t batch, int32_t G, int32_t max_seq_len, int64_t total_rows,
@@ -284,7 +291,8 @@ gqa_status plan_impl(int32_t batch, int32_t G, int32_t max_seq_len, int64_t tota
     const int64_t rem = ctas % resident;
     const double waves = static_cast<double>(ctas / resident) +
                          (rem ? static_cast<double>(std::max<int64_t>(rem, sm_count)) / resident : 0.0);
-    const double cost = waves * static_cast<double>(chunk + 128) + 4.0 * S;
+    const double merge = (S > 1 && N >= 2048) ? 256.0 : 0.0;
+    const double cost = waves * static_cast<double>(chunk + 128) + 4.0 * S + merge;
     if (best_splits == 0 || cost < best) {
       best = cost;
       best_chunk = chunk;
