@@ -304,6 +304,11 @@ class Op:
             self.vcodes = torch.roll(code, 1, 0).to(dev).contiguous()
             self.atoms = torch.nn.functional.normalize(torch.randn((n_atoms, D), generator=cg), dim=1).to(dev)
             self.kv_bytes = 2 * self.kcodes.numel() * 4
+            # the codes are small: enough copies, taken in turn, that each
+            # step's codes come from HBM (more than twice the L2 in all)
+            ncopy = min(16, max(2, -(-2 * 126_000_000 // self.kv_bytes)))
+            self.code_sets = [(self.kcodes, self.vcodes)] + [
+                (self.kcodes.clone(), self.vcodes.clone()) for _ in range(ncopy - 1)]
             self.kernel = "gqa_partition_coded_kernel"
         # the split plan of the plain call, and the three-call path's buffers
         self.S_ws, self.S, self.chunk = gqa.gqa_decode_workspace_size(
@@ -326,7 +331,8 @@ class Op:
         common = dict(score_scale=w.score_scale, max_seq_len=w.max_seq_len, workspace=self.ws, stream=st,
                       flags=fl)
         if self.op == "coded_attend":
-            gqa.gqa_decode_attend_coded(self.q, self.kcodes, self.vcodes, self.atoms, self.atoms, self.offsets,
+            kc, vc = self.code_sets[i % len(self.code_sets)]
+            gqa.gqa_decode_attend_coded(self.q, kc, vc, self.atoms, self.atoms, self.offsets,
                                         H, G, carry=self.carry, out=self.out, num_splits=self.forced, **common)
         elif self.op == "append_attend":
             gqa.gqa_decode_append_attend(self.q, k, v, self.offsets, self.k_new, self.v_new, H, G,
@@ -350,6 +356,13 @@ class Op:
         gqa, w = self.gqa, self.w
         if not hasattr(self, "parts_only"):
             self.parts_only = gqa.State.empty(w.batch * w.num_heads, w.head_dim, self.q.device, (self.S,))
+        if self.op == "coded_attend":
+            kc, vc = self.code_sets[i % len(self.code_sets)]
+            gqa.gqa_decode_attend_coded(self.q, kc, vc, self.atoms, self.atoms, self.offsets, w.num_heads,
+                                        w.num_kv_heads, score_scale=w.score_scale, partials_out=self.parts_only,
+                                        num_splits=self.S, max_seq_len=w.max_seq_len, workspace=self.ws,
+                                        stream=st)
+            return
         k, v = self.caches[i % len(self.caches)]
         gqa.gqa_decode_attend(self.q, k, v, self.offsets, w.num_heads, w.num_kv_heads,
                               score_scale=w.score_scale, partials_out=self.parts_only, num_splits=self.S,
@@ -580,7 +593,9 @@ def run_ours(args):
                 "num_heads": H, "num_kv_heads": w.num_kv_heads, "head_dim": D, "seq_len": w.max_seq_len,
                 "total_rows": w.total_rows, "kv_bytes_per_step": kv_bytes, "num_splits": op.S,
                 "chunk_len": op.chunk,
-                "l2": (f"inputs larger than L2: {len(op.caches)} cache copies of "
+                "l2": (f"inputs larger than L2: {len(op.code_sets)} copies of the {kv_bytes / 2**20:.0f} MiB "
+                       f"of codes taken in turn" if args.op == "coded_attend" else
+                       f"inputs larger than L2: {len(op.caches)} cache copies of "
                        f"{kv_bytes / 2**20:.0f} MiB alternated" if len(op.caches) > 1 else
                        f"inputs larger than L2: one {kv_bytes / 2**20:.0f} MiB cache, > 4x the 126 MB L2"),
                 "parallelism": f"replicas x{world} (independent batches, no collective)",

@@ -44,16 +44,13 @@ constexpr int kCodedMaxRoundKeys = 8192;
 // words, after the header:
 //   ring    P x W x 512: a thread's next P code rows (P = 4, 2 or 1, as many
 //           as fit with a round of 512 keys);
-//   round   KR x (V + hpk + 1): up to 8 words per row (V = W), the round's V
-//           code rows (above 8, V = 0: V rows pass through the ring twice
-//           instead); its logits (then weights) and |V coefficient| sums. KR
+//   round   KR x (hpk + 1): the round's logits and |V coefficient| sums, KR
 //           keys, a multiple of 512, at most 8192, as many as fit. The round
 //           region also stages atom rows;
 //   tables  3 x hpk x n_atoms: logit table, value weights, round weights.
-__host__ __device__ constexpr int coded_vstore_words(int words) { return 0 * words; }
 __host__ __device__ constexpr int coded_table_words(int hpk, int n_atoms) { return 3 * hpk * n_atoms; }
 __host__ __device__ constexpr int coded_free_words() { return (kCodedSmemBudget - kCodedFixedBytes) / 4; }
-__host__ __device__ constexpr int coded_key_words(int words, int hpk) { return coded_vstore_words(words) + hpk + 1; }
+__host__ __device__ constexpr int coded_key_words(int words, int hpk) { return 0 * words + hpk + 1; }
 __host__ __device__ constexpr bool coded_ring_fits(int rows, int words, int hpk, int n_atoms) {
   return rows * words * kCodedThreads + kCodedThreads * coded_key_words(words, hpk) +
              coded_table_words(hpk, n_atoms) <=
@@ -129,23 +126,24 @@ __device__ __forceinline__ void cta_reduce_heads(const float (*v)[NW], int hpk, 
 // value epilogue (threads own 4 columns of one head for a share of the atoms,
 // then the shares add in a fixed order).
 // Keys go in rounds of KR (a multiple of 512); thread tid takes keys tid, tid
-// + 512, ... of a round. Its K code rows pass through its own P-row ring and
-// its V code rows land in its own slots of the round's V store (cp.async, the
-// next round's copies issued as soon as the thread is done with the current
-// one's rows, so they run across the barriers; no thread touches another's
-// slots); rows above 8 words, whose V store would not fit beside the largest
-// tables, instead pass through the ring again for passes B and C. Per round,
-// three passes and two barriers:
-//   A. logits by table lookups into the round's logit store, each key's sum of
-//      |V coefficient| from its V row, the warps' maxima per head -> barrier;
-//   B. the new running maximum; the last round's integer weights folded into
-//      Wt, both rescaled to it; each key's weights p (over its logits in the
-//      store), the partition, and per head the bound sum_j p_j sum_w |c'_jw|
-//      on any atom's weight sum -> barrier;
-//   C. every weight p * c' added to the integer table Wb in fixed point,
-//      scaled by a power of two that keeps the bound below 2^30 (32-bit
-//      shared atomics, which B200 runs several times faster than float ones,
-//      and whose sums do not depend on their order).
+// + 512, ... of a round. Its code rows pass through its own P-row ring
+// (cp.async; no thread touches another's slots, and the next pass's first rows
+// are issued before each barrier, so they run across it). Per round, two
+// passes and one barrier between them:
+//   A. the K and V rows of each key in turn: logits by table lookups into the
+//      round's logit store, each key's sum of |V coefficient|, and the
+//      thread's maxima per head; then, out of its own keys' entries of the
+//      store, its share of the bound sum_j p_j sum_w |c'_jw| on any atom's
+//      weight sum, relative to its own maxima. The warps combine (maximum,
+//      bound) pairs -> barrier;
+//   C. the new running maximum and the round's bound relative to it; each
+//      key's weights p, the partition, and every weight p * c' added to the
+//      integer table Wb in fixed point, scaled by a power of two that keeps
+//      the bound below 2^30 (32-bit shared atomics, which B200 runs several
+//      times faster than float ones, and whose sums do not depend on their
+//      order).
+// After a barrier each thread folds its atoms of Wb into the value weights Wt,
+// both rescaled to the new running maximum, and clears them.
 // Cross-warp maxima and sums go through a fixed-order lane butterfly, so the
 // results are bit-reproducible. A segment with one split (the tile is the
 // whole sequence) folds the carry and writes out / state_out directly; others
@@ -156,11 +154,12 @@ __global__ void __launch_bounds__(kCodedThreads, 1)
 gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   static_assert(MW == 4 || MW == 8 || MW == 16, "words bound 4, 8 or 16");
   constexpr int NT = kCodedThreads, NW = NT / 32, E = D / 32;
-  constexpr bool VST = MW < 0;           // V rows kept in the round's store (else streamed twice)
   extern __shared__ uint8_t dsm_raw[];
-  uint32_t* dsm = reinterpret_cast<uint32_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
+  // aligned by an offset from the array itself, so that every access through
+  // these pointers stays a shared-memory access for the compiler
+  uint32_t* dsm = reinterpret_cast<uint32_t*>(dsm_raw + ((128u - (ptx::smem_u32(dsm_raw) & 127u)) & 127u));
   __shared__ float red[HMAX][NW];        // per head, per warp: maxima (then partitions)
-  __shared__ float red2[2][HMAX][NW];    // per head, per warp: weight bounds, by round parity
+  __shared__ float red2[HMAX][NW];       // per head, per warp: weight bounds
   __shared__ float smM[16], smL[16], smC[16];
   __shared__ float hM[16], hL[16];       // per head: base-2 running maximum, partition
   __shared__ int smFlag;
@@ -171,8 +170,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   const uint32_t bar0 = ptx::smem_u32(dsm);                    // atom copies into buffer 0 / 1
   const uint32_t bar1 = bar0 + 8;
   uint32_t* ring = dsm + 64;                                   // [P][W or W/4 quads][NT] K rows
-  uint32_t* vst = ring + P * W * NT;                           // [W or W/4 quads][KR] V rows (VST)
-  float* lg = reinterpret_cast<float*>(vst + (VST ? KR * W : 0));   // [KR][hpk] logits, then weights
+  float* lg = reinterpret_cast<float*>(ring + P * W * NT);    // [KR][hpk] logits
   float* cs = lg + KR * hpk;                                   // [KR] sums of |V coefficient|
   float* qa = cs + KR;                                         // [NA][hpk] logits (base 2)
   float* Wt = qa + hpk * NA;                                   // [hpk][NA] value weights
@@ -200,21 +198,47 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   auto round_keys = [&](int rd) { return min(KR, t.kend - t.kbeg - rd * KR); };
   auto rows_of = [&](int nk) { return nk > tid ? (nk - tid + NT - 1) / NT : 0; };
 
-  // ---- code rows
-  const uint32_t ring_u32 = ptx::smem_u32(ring), vst_u32 = ptx::smem_u32(vst);
-  auto copy_row = [&](uint32_t dst, int step, const uint32_t* src) {   // step: bytes between quads / words
+  // ---- code rows: a stream of rows through the ring's P slots, one commit
+  // group per row (empty past the stream's end), row n of a stream in slot
+  // n % P. Pass A's stream is the K and V rows of this thread's keys in turn
+  // (K, V of key tid, then of key tid + NT, ...), pass C's its V rows. A
+  // slot is refilled only after the row read out of it has been used.
+  const uint32_t ring_u32 = ptx::smem_u32(ring);
+  auto copy_row = [&](uint32_t dst, const uint32_t* src) {
     if (quads) {
-      for (int q = 0; q < W / 4; ++q) ptx::cp_async_16(dst + q * step, src + 4 * q);
+      for (int q = 0; q < W / 4; ++q) ptx::cp_async_16(dst + q * NT * 16, src + 4 * q);
     } else {
-      for (int w = 0; w < W; ++w) ptx::cp_async_4(dst + w * step, src + w);
+      for (int w = 0; w < W; ++w) ptx::cp_async_4(dst + w * NT * 4, src + w);
     }
   };
-  auto read_row = [&](const uint32_t* base, int stride, uint32_t (&r)[MW]) {   // stride: quads / words
+  // row n of the round starting at key kb with `mine` keys of this thread:
+  // pass A (two rows a key) or pass C (V rows)
+  auto issue = [&](bool pass_a, int kb, int mine, int n) {
+    const int i = pass_a ? n >> 1 : n;
+    if (i < mine) {
+      const int sl = n % P;
+      const uint32_t* base = (pass_a && (n & 1) == 0) ? kbase : vbase;
+      copy_row(ring_u32 + (quads ? (sl * (W / 4) * NT + tid) * 16 : (sl * W * NT + tid) * 4),
+               base + static_cast<size_t>(kb + tid + i * NT) * row_stride);
+    }
+    ptx::cp_async_commit();
+  };
+  auto prime = [&](bool pass_a, int kb, int mine) {
+    for (int n = 0; n < P; ++n) issue(pass_a, kb, mine, n);
+  };
+  auto fetch = [&](int n, uint32_t (&r)[MW]) {   // wait for row n, read it
+    if (P >= 4)
+      ptx::cp_async_wait_group<3>();
+    else if (P == 2)
+      ptx::cp_async_wait_group<1>();
+    else
+      ptx::cp_async_wait_group<0>();
+    const uint32_t* base = ring + (quads ? ((n % P) * (W / 4) * NT + tid) * 4 : (n % P) * W * NT + tid);
     if (quads) {
 #pragma unroll
       for (int q = 0; q < MW / 4; ++q) {
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (4 * q < W) v = reinterpret_cast<const uint4*>(base)[q * stride];
+        if (4 * q < W) v = reinterpret_cast<const uint4*>(base)[q * NT];
         r[4 * q] = v.x;
         r[4 * q + 1] = v.y;
         r[4 * q + 2] = v.z;
@@ -222,50 +246,10 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       }
     } else {
 #pragma unroll
-      for (int w = 0; w < MW; ++w) r[w] = w < W ? base[w * stride] : 0u;
+      for (int w = 0; w < MW; ++w) r[w] = w < W ? base[w * NT] : 0u;
     }
   };
-  // Row i of this thread's keys of `base` in the round starting at kb into ring
-  // slot i % P (one commit group, empty past its rows)
-  auto issue_row = [&](const uint32_t* base, int kb, int mine, int i) {
-    if (i < mine) {
-      const int sl = i % P;
-      copy_row(ring_u32 + (quads ? (sl * (W / 4) * NT + tid) * 16 : (sl * W * NT + tid) * 4),
-               quads ? NT * 16 : NT * 4, base + static_cast<size_t>(kb + tid + i * NT) * row_stride);
-    }
-    ptx::cp_async_commit();
-  };
-  auto prime = [&](const uint32_t* base, int kb, int mine) {
-    for (int i = 0; i < P; ++i) issue_row(base, kb, mine, i);
-  };
-  auto wait_ring = [&] {             // the oldest of the P rows in flight has landed
-    if (P >= 4)
-      ptx::cp_async_wait_group<3>();
-    else if (P == 2)
-      ptx::cp_async_wait_group<1>();
-    else
-      ptx::cp_async_wait_group<0>();
-  };
-  auto ring_row = [&](int i, uint32_t (&r)[MW]) {
-    const int sl = i % P;
-    read_row(ring + (quads ? (sl * (W / 4) * NT + tid) * 4 : sl * W * NT + tid), NT, r);
-  };
-  // A round's copies: with the V store, this thread's V rows (one group,
-  // older than every K row of the round, so a K row that has landed means they
-  // have too); then its first P K rows.
-  auto start_round = [&](int rd) {
-    const int kb = t.kbeg + rd * KR, nk = round_keys(rd), mine = rows_of(nk);
-    if (VST) {
-      for (int i = 0; i < mine; ++i) {
-        const int j = tid + i * NT;
-        copy_row(vst_u32 + (quads ? j * 16 : j * 4), quads ? KR * 16 : KR * 4,
-                 vbase + static_cast<size_t>(kb + j) * row_stride);
-      }
-      ptx::cp_async_commit();
-    }
-    prime(kbase, kb, mine);
-  };
-  if (nround > 0) start_round(0);
+  if (nround > 0) prime(true, t.kbeg, rows_of(round_keys(0)));
 
   // ---- atom rows: chunks of `chunk` atoms through two buffers in the logit
   // store region, by bulk copies completing on bar0 / bar1. A chunk's copy is
@@ -336,19 +320,25 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
     constexpr int HT = HMAX > 8 ? 8 : HMAX;
     constexpr int A = 32 / HT;
     const size_t qrow = static_cast<size_t>(t.b) * a.H + static_cast<size_t>(t.g) * hpk;
+    // this lane's columns of HT query heads from h0; the first HT are loaded
+    // before the atom copies are waited for, and kept when they are all
+    float qreg[HT][E];
+    auto load_q = [&](int h0) {
+#pragma unroll
+      for (int h = 0; h < HT; ++h)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const size_t qi = (qrow + h0 + h) * D + lane * E + e;
+          qreg[h][e] = h0 + h >= hpk ? 0.f
+                       : c.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qi])
+                                  : static_cast<const float*>(a.q)[qi];
+        }
+    };
+    load_q(0);
     over_atoms(c.k_atoms, abuf, region, [&](int c0, int n, const float* rows) {
 #pragma unroll 1
       for (int h0 = 0; h0 < hpk; h0 += HT) {
-        float qreg[HT][E];
-#pragma unroll
-        for (int h = 0; h < HT; ++h)
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            const size_t qi = (qrow + h0 + h) * D + lane * E + e;
-            qreg[h][e] = h0 + h >= hpk ? 0.f
-                         : c.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qi])
-                                    : static_cast<const float*>(a.q)[qi];
-          }
+        if (hpk > HT) load_q(h0);
         for (int a0 = warp * A; a0 < n; a0 += NW * A) {
           float v[32];
 #pragma unroll
@@ -393,35 +383,66 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   }
   __syncthreads();                   // the table is complete; the logit store is free
 
-  // running maximum per head (identical in every thread) and this thread's
-  // share of the partition; the bounds of the last round stay in red2
-  // (double-buffered by round parity) for its fold.
+  // Running maximum per head (identical in every thread) and this thread's
+  // share of the partition. Per round, one barrier between the passes:
+  //   A. K rows: logits by table lookup into lg[key][h] and this thread's
+  //      maxima; V rows: the sum of |coefficient| of each key into cs. Then,
+  //      from its own keys in shared memory, the thread's share of the bound
+  //      sum_j p_j sum_w |c'_jw| relative to its own maxima. Warps combine
+  //      (maximum, bound) pairs -> barrier;
+  //   C. the round's maximum and bound from the warps' pairs in a fixed order;
+  //      weights p, the partition, and the weights into Wb in fixed point.
+  // After a barrier, each thread folds its atoms of Wb into Wt (both rescaled
+  // to the new running maximum) and clears them.
   float mrun[HMAX], lthr[HMAX];
 #pragma unroll
   for (int h = 0; h < HMAX; ++h) {
     mrun[h] = -INFINITY;
     lthr[h] = 0.f;
   }
-  auto fmax_op = [](float x, float y) { return fmaxf(x, y); };
+  // (maximum, bound) pairs: the bound rescaled to the larger maximum; the
+  // combination is symmetric, so a butterfly leaves the same bits in every lane
+  auto pair_combine = [](float& m, float& s, float m2, float s2) {
+    const float mm = fmaxf(m, m2);
+    const float a = m == -INFINITY ? 0.f : s * exp2f(m - mm);
+    const float b = m2 == -INFINITY ? 0.f : s2 * exp2f(m2 - mm);
+    m = mm;
+    s = a + b;
+  };
   auto fadd_op = [](float x, float y) { return x + y; };
   bool bad = false;
   const bool quad_heads = (hpk & 3) == 0;
+  auto load_heads = [&](const float* src, float (&x)[HMAX]) {
+    if (quad_heads) {
+#pragma unroll
+      for (int q4 = 0; q4 < HMAX / 4; ++q4)
+        if (4 * q4 < hpk) {
+          const float4 t4 = *reinterpret_cast<const float4*>(src + 4 * q4);
+          x[4 * q4] = t4.x;
+          x[4 * q4 + 1] = t4.y;
+          x[4 * q4 + 2] = t4.z;
+          x[4 * q4 + 3] = t4.w;
+        }
+    } else {
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h)
+        if (h < hpk) x[h] = src[h];
+    }
+  };
 #pragma unroll 1
   for (int rd = 0; rd < nround && ok; ++rd) {
-    const int par = rd & 1;
     const int kb = t.kbeg + rd * KR;
     const int nk = round_keys(rd);
     const int mine = rows_of(nk);
-    // ---- pass A: logits by table lookup into lg[key][h]; |V coefficient| sums
+    // ---- pass A
     float tmax[HMAX];
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) tmax[h] = -INFINITY;
 #pragma unroll 1
     for (int i = 0; i < mine; ++i) {
-      wait_ring();
       const int j = tid + i * NT;
       uint32_t kw[MW];
-      ring_row(i, kw);
+      fetch(2 * i, kw);
       float s[HMAX];
 #pragma unroll
       for (int h = 0; h < HMAX; ++h) s[h] = 0.f;
@@ -450,14 +471,14 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
             if (h < hpk) s[h] = fmaf(cf, row[h], s[h]);
         }
       }
-      if (VST) {
-        uint32_t vw[MW];
-        read_row(vst + (quads ? j * 4 : j), KR, vw);
-        float csum = 0.f;
+      issue(true, kb, mine, 2 * i + P);          // the K row's slot is free
+      uint32_t vw[MW];
+      fetch(2 * i + 1, vw);
+      float csum = 0.f;                          // sum of |V coefficient| of the key
 #pragma unroll
-        for (int w = 0; w < MW; ++w) csum += fabsf(code_coeff(vw[w]));
-        cs[j] = csum;
-      }
+      for (int w = 0; w < MW; ++w) csum += fabsf(code_coeff(vw[w]));
+      issue(true, kb, mine, 2 * i + 1 + P);      // the V row's slot is free
+      cs[j] = csum;
       const float bb = bias2(a, t, kb + j);
       float* dst = lg + j * hpk;
       if (quad_heads) {
@@ -473,136 +494,105 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       }
 #pragma unroll
       for (int h = 0; h < HMAX; ++h) tmax[h] = fmaxf(tmax[h], s[h] + bb);
-      issue_row(kbase, kb, mine, i + P);   // the slot's row has been used: refill it
     }
-    if (!VST) prime(vbase, kb, mine);  // pass B's V rows come in across the barrier
+    prime(false, kb, mine);          // pass C's V rows come in across the barrier
+    // this thread's bound relative to its own maxima, from its keys' logits
+    // and coefficient sums (no copy involved)
+    float tb[HMAX];
 #pragma unroll
-    for (int h = 0; h < HMAX; ++h) {
-      if (h >= hpk) break;
-      float v = tmax[h];
-#pragma unroll
-      for (int x = 16; x >= 1; x >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, x));
-      if (lane == 0) red[h][warp] = v;
-    }
-    __syncthreads();                 // red complete; the last round's atomics done
-    // ---- pass B: new maximum; fold of the last round's Wb into Wt; weights
-    // p into lg; partition; bound on any atom's weight sum
-    float mn[HMAX];
-    cta_reduce_heads<HMAX, NW>(red, hpk, lane, -INFINITY, mn, fmax_op);
-    {
-      float unit[HMAX];
-      if (rd > 0) cta_reduce_heads<HMAX, NW>(red2[par ^ 1], hpk, lane, 0.f, unit, fadd_op);
-#pragma unroll
-      for (int h = 0; h < HMAX; ++h) {
-        if (h >= hpk) break;
-        mn[h] = fmaxf(mrun[h], mn[h]);
-        const float f = (mn[h] == -INFINITY) ? 1.f : exp2f(mrun[h] - mn[h]);
-        mrun[h] = mn[h];
-        lthr[h] *= f;
-        if (rd > 0) {
-          // Wt and the last round's Wb are both relative to the previous
-          // maximum: add them and rescale to the new one; clear Wb
-          const float sc = block_weight_scale(unit[h]);
-          const float u = sc > 0.f ? 1.f / sc : 0.f;
-          for (int i = h * NA + tid; i < (h + 1) * NA; i += NT) {
-            Wt[i] = (Wt[i] + static_cast<float>(static_cast<int32_t>(Wb[i])) * u) * f;
-            Wb[i] = 0u;
-          }
-        }
-        if (mn[h] == -INFINITY) mn[h] = 0.f;          // all masked so far: weights 0
-      }
-    }
-    float bnd[HMAX];
-#pragma unroll
-    for (int h = 0; h < HMAX; ++h) bnd[h] = 0.f;
+    for (int h = 0; h < HMAX; ++h) tb[h] = 0.f;
 #pragma unroll 2
     for (int i = 0; i < mine; ++i) {
       const int j = tid + i * NT;
-      float csum;
-      if (VST) {
-        csum = cs[j];
-      } else {
-        wait_ring();
-        uint32_t vw[MW];
-        ring_row(i, vw);
-        csum = 0.f;
-#pragma unroll
-        for (int w = 0; w < MW; ++w) csum += fabsf(code_coeff(vw[w]));
-        issue_row(vbase, kb, mine, i + P);
-      }
-      float* src = lg + j * hpk;
+      float l[HMAX];
+      load_heads(lg + j * hpk, l);
+      const float c = cs[j];
 #pragma unroll
       for (int h = 0; h < HMAX; ++h)
-        if (h < hpk) {
-          const float p = exp2f(src[h] - mn[h]);
-          src[h] = p;
-          lthr[h] += p;
-          bnd[h] = fmaf(p, csum, bnd[h]);
-        }
+        if (h < hpk && tmax[h] != -INFINITY) tb[h] = fmaf(exp2f(l[h] - tmax[h]), c, tb[h]);
     }
-    if (!VST) prime(vbase, kb, mine);  // pass C's V rows come in across the barrier
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
       if (h >= hpk) break;
-      float v = bnd[h];
+      float m = tmax[h], sb = tb[h];
 #pragma unroll
-      for (int x = 16; x >= 1; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
-      if (lane == 0) red2[par][h][warp] = v;
+      for (int x = 16; x >= 1; x >>= 1)
+        pair_combine(m, sb, __shfl_xor_sync(0xffffffffu, m, x), __shfl_xor_sync(0xffffffffu, sb, x));
+      if (lane == 0) {
+        red[h][warp] = m;
+        red2[h][warp] = sb;
+      }
     }
-    __syncthreads();                 // red2 complete; Wb folded and clear
-    // ---- pass C: the weights into Wb, in fixed point
-    float scale[HMAX];
-    cta_reduce_heads<HMAX, NW>(red2[par], hpk, lane, 0.f, scale, fadd_op);
+    __syncthreads();                 // red, red2 complete
+    // ---- pass C
+    float mn[HMAX], scale[HMAX], fr[HMAX];
 #pragma unroll
-    for (int h = 0; h < HMAX; ++h) scale[h] = h < hpk ? block_weight_scale(scale[h]) : 0.f;
+    for (int h = 0; h < HMAX; ++h) {
+      mn[h] = 0.f;
+      scale[h] = 0.f;
+      fr[h] = 1.f;
+      if (h >= hpk) continue;
+      float m = lane < NW ? red[h][lane] : -INFINITY;
+      float sb = lane < NW ? red2[h][lane] : 0.f;
+#pragma unroll
+      for (int x = 16; x >= 1; x >>= 1)
+        pair_combine(m, sb, __shfl_xor_sync(0xffffffffu, m, x), __shfl_xor_sync(0xffffffffu, sb, x));
+      const float mnew = fmaxf(mrun[h], m);
+      fr[h] = (mnew == -INFINITY) ? 1.f : exp2f(mrun[h] - mnew);
+      mrun[h] = mnew;
+      lthr[h] *= fr[h];
+      // weights relative to the running maximum are at most those relative
+      // to the round's, so the round's bound still bounds them
+      scale[h] = block_weight_scale(m == -INFINITY ? 0.f : sb * exp2f(m - mnew));
+      mn[h] = mnew == -INFINITY ? 0.f : mnew;    // all masked so far: weights 0
+    }
 #pragma unroll 1
     for (int i = 0; i < mine; ++i) {
       const int j = tid + i * NT;
       uint32_t vw[MW];
-      if (VST) {
-        read_row(vst + (quads ? j * 4 : j), KR, vw);
-      } else {
-        wait_ring();
-        ring_row(i, vw);
-      }
-      float ps[HMAX];                // weights in fixed-point units
-      const float* src = lg + j * hpk;
+      fetch(i, vw);
+      float l[HMAX], ps[HMAX];       // weights in fixed-point units
+      load_heads(lg + j * hpk, l);
 #pragma unroll
-      for (int h = 0; h < HMAX; ++h) ps[h] = h < hpk ? src[h] * scale[h] : 0.f;
+      for (int h = 0; h < HMAX; ++h) {
+        ps[h] = 0.f;
+        if (h < hpk) {
+          const float p = exp2f(l[h] - mn[h]);
+          lthr[h] += p;
+          ps[h] = p * scale[h];
+        }
+      }
+      // every word adds its weights, zero ones included (no branch); an index
+      // out of range is flagged and adds zeros to atom 0
 #pragma unroll
       for (int w = 0; w < MW; ++w) {
+        if (w >= W) break;
         const int idx = static_cast<int>(vw[w] >> 16);
-        const float cf = code_coeff(vw[w]);
         const bool in = idx < NA;
         bad |= !in;
-        if (!in || cf == 0.f) continue;
-        uint32_t* wrow = Wb + idx;
+        const float cf = in ? code_coeff(vw[w]) : 0.f;
+        uint32_t* wrow = Wb + (in ? idx : 0);
 #pragma unroll
         for (int h = 0; h < HMAX; ++h)
-          if (h < hpk && ps[h] != 0.f)
-            atomicAdd(wrow + h * NA, static_cast<uint32_t>(__float2int_rn(ps[h] * cf)));
+          if (h < hpk) atomicAdd(wrow + h * NA, static_cast<uint32_t>(__float2int_rn(ps[h] * cf)));
       }
-      if (!VST) issue_row(vbase, kb, mine, i + P);
+      issue(false, kb, mine, i + P);
     }
-    // this thread is done with its rows of the round: the next round's copies
-    // start now, across the barrier
-    if (rd + 1 < nround) start_round(rd + 1);
-  }
-  ptx::cp_async_wait_group<0>();     // no copy left in flight
-  __syncthreads();                   // the last round's atomics done
-  // the last round's weights
-  if (nround > 0 && ok) {
-    float unit[HMAX];
-    cta_reduce_heads<HMAX, NW>(red2[(nround - 1) & 1], hpk, lane, 0.f, unit, fadd_op);
+    // the next round's rows start coming in across the barrier
+    if (rd + 1 < nround) prime(true, kb + KR, rows_of(round_keys(rd + 1)));
+    __syncthreads();                 // the round's atomics done
+    // fold: Wt and Wb relative to the new running maximum; Wb cleared
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
       if (h >= hpk) break;
-      const float sc = block_weight_scale(unit[h]);
-      const float u = sc > 0.f ? 1.f / sc : 0.f;
-      for (int i = h * NA + tid; i < (h + 1) * NA; i += NT)
-        Wt[i] += static_cast<float>(static_cast<int32_t>(Wb[i])) * u;
+      const float u = scale[h] > 0.f ? 1.f / scale[h] : 0.f;
+      for (int i = h * NA + tid; i < (h + 1) * NA; i += NT) {
+        Wt[i] = fmaf(Wt[i], fr[h], static_cast<float>(static_cast<int32_t>(Wb[i])) * u);
+        Wb[i] = 0u;
+      }
     }
   }
+  ptx::cp_async_wait_group<0>();     // no copy left in flight
   // the partition: every thread's share, summed in a fixed order
 #pragma unroll
   for (int h = 0; h < HMAX; ++h) {

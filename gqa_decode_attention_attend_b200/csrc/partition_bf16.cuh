@@ -51,7 +51,9 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const PartitionArgs a) {
   using C = TcCfg<D, NT>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by an offset from the array itself (the compiler keeps accesses
+  // through it in the shared state space)
+  uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t ring = ptx::smem_u32(smem);
   const uint32_t bar_full = ring + C::kBarOffset;
   const uint32_t bar_empty = bar_full + C::kStages * 8;

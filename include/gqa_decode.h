@@ -236,12 +236,14 @@ typedef struct {
  * per-atom weights applied to the V atoms once). params->k, ->v and ->kv_dtype
  * are ignored; q is fp32 or bf16; everything else (offsets, carry, bias,
  * partials, outputs, workspace, flags) as gqa_decode_attend. A code word naming
- * an atom >= n_atoms is skipped and flags GQA_ERR_BAD_CODES in the device error
- * word. The per-atom value weights are summed per super-block of 512 or 1024
- * keys in 32-bit fixed point, scaled to the super-block's largest possible sum
- * (rounding error at most 2^-31 of it per weight), so results are
- * bit-reproducible. The split plan is the coded kernel's own (one CTA of 512
- * threads per SM), so size the workspace with gqa_decode_coded_workspace_size. */
+ * an atom >= n_atoms contributes nothing and flags GQA_ERR_BAD_CODES in the
+ * device error word. The per-atom value weights are summed per round of keys (a
+ * multiple of 512, at most 8192, as many as shared memory holds) in 32-bit fixed
+ * point, scaled by a power of two to the round's largest possible sum
+ * sum_j p_j sum_w |coeff_jw| (rounding error at most 2^-31 of it per weight), so
+ * results are bit-reproducible. The split plan is the coded kernel's own (one
+ * CTA of 512 threads per SM), so size the workspace with
+ * gqa_decode_coded_workspace_size. */
 gqa_status gqa_decode_attend_coded(const gqa_decode_params* params, const gqa_kv_codes* codes,
                                    gqa_stream_t stream);
 
