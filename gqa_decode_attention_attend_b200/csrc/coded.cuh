@@ -196,49 +196,75 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   const uint32_t* kbase = c.k_codes + (static_cast<size_t>(t.o0) * a.G + t.g) * W;
   const uint32_t* vbase = c.v_codes + (static_cast<size_t>(t.o0) * a.G + t.g) * W;
   auto round_keys = [&](int rd) { return min(KR, t.kend - t.kbeg - rd * KR); };
-  auto rows_of = [&](int nk) { return nk > tid ? (nk - tid + NT - 1) / NT : 0; };
+  // keys of a round in warp w's rows: tid + i * NT for i < rows_of(nk), the
+  // count of the warp's lane 0 (the most in the warp), so that loops over a
+  // warp's rows run the same count in every lane; a lane whose key is past the
+  // round (j >= nk) takes part in the copies and warp syncs and nothing else
+  auto rows_of = [&](int nk) { return nk > warp * 32 ? (nk - warp * 32 + NT - 1) / NT : 0; };
 
   // ---- code rows: a stream of rows through the ring's P slots, one commit
   // group per row (empty past the stream's end), row n of a stream in slot
-  // n % P. Pass A's stream is the K and V rows of this thread's keys in turn
-  // (K, V of key tid, then of key tid + NT, ...), pass C's its V rows. A
-  // slot is refilled only after the row read out of it has been used.
+  // n % P. Pass A's stream is the K and V rows of the thread's keys in turn
+  // (K, V of key tid, then of key tid + NT, ...), pass C's its V rows. Each
+  // warp's part of a slot holds its 32 keys' rows ([32][W] words), copied by
+  // the lanes together: 16-byte units u = lane + 32 k (quad u % QR of row
+  // u / QR, QR = W / 4), so that a copy instruction reads whole 32-byte
+  // sectors; quad q of row r sits at q ^ ((r >> s) & (QR - 1)) when QR is a
+  // power of two (8 >> s = 8 / QR rows a 128-byte line), which keeps each lane's
+  // reads of its own row free of bank conflicts. Rows of W not a multiple of
+  // 4 are copied word by word, each lane its own. A warp sync after the wait
+  // makes the lanes' copies visible to the warp, and one before each copy
+  // keeps it off a row that a lane still reads.
   const uint32_t ring_u32 = ptx::smem_u32(ring);
-  auto copy_row = [&](uint32_t dst, const uint32_t* src) {
-    if (quads) {
-      for (int q = 0; q < W / 4; ++q) ptx::cp_async_16(dst + q * NT * 16, src + 4 * q);
-    } else {
-      for (int w = 0; w < W; ++w) ptx::cp_async_4(dst + w * NT * 4, src + w);
-    }
-  };
-  // row n of the round starting at key kb with `mine` keys of this thread:
-  // pass A (two rows a key) or pass C (V rows)
-  auto issue = [&](bool pass_a, int kb, int mine, int n) {
+  const int QR = W / 4;
+  const bool qswz = quads && (QR & (QR - 1)) == 0;
+  const int qsh = QR == 4 ? 1 : (QR == 2 ? 2 : 3);
+  auto qpos = [&](int q, int r) { return qswz ? (q ^ ((r >> qsh) & (QR - 1))) : q; };
+  int u_row[MW / 4], u_src[MW / 4], u_dst[MW / 4];   // this lane's units: row, source and slot words
+#pragma unroll
+  for (int k = 0; k < MW / 4; ++k) {
+    const int u = lane + 32 * k;
+    u_row[k] = quads ? u / max(QR, 1) : 32;
+    const int q = quads ? u % max(QR, 1) : 0;
+    u_src[k] = u_row[k] * static_cast<int>(a.G) * W + 4 * q;
+    u_dst[k] = u_row[k] * W + 4 * qpos(q, u_row[k]);
+  }
+  // row n of the round starting at key kb with nk keys: pass A (two rows a
+  // key) or pass C (V rows)
+  auto issue = [&](bool pass_a, int kb, int nk, int n) {
+    __syncwarp();
     const int i = pass_a ? n >> 1 : n;
-    if (i < mine) {
-      const int sl = n % P;
-      const uint32_t* base = (pass_a && (n & 1) == 0) ? kbase : vbase;
-      copy_row(ring_u32 + (quads ? (sl * (W / 4) * NT + tid) * 16 : (sl * W * NT + tid) * 4),
-               base + static_cast<size_t>(kb + tid + i * NT) * row_stride);
+    const int j0 = warp * 32 + i * NT;             // the warp's first key of the step
+    if (j0 < nk) {
+      const uint32_t dst = ring_u32 + ((n % P) * NW + warp) * 32 * W * 4;
+      const uint32_t* src = ((pass_a && (n & 1) == 0) ? kbase : vbase) + static_cast<size_t>(kb + j0) * row_stride;
+      if (quads) {
+#pragma unroll
+        for (int k = 0; k < MW / 4; ++k)
+          if (k < QR && j0 + u_row[k] < nk) ptx::cp_async_16(dst + u_dst[k] * 4, src + u_src[k]);
+      } else if (j0 + lane < nk) {
+        for (int w = 0; w < W; ++w) ptx::cp_async_4(dst + (lane * W + w) * 4, src + lane * row_stride + w);
+      }
     }
     ptx::cp_async_commit();
   };
-  auto prime = [&](bool pass_a, int kb, int mine) {
-    for (int n = 0; n < P; ++n) issue(pass_a, kb, mine, n);
+  auto prime = [&](bool pass_a, int kb, int nk) {
+    for (int n = 0; n < P; ++n) issue(pass_a, kb, nk, n);
   };
-  auto fetch = [&](int n, uint32_t (&r)[MW]) {   // wait for row n, read it
+  auto fetch = [&](int n, uint32_t (&r)[MW]) {   // wait for row n, read this lane's
     if (P >= 4)
       ptx::cp_async_wait_group<3>();
     else if (P == 2)
       ptx::cp_async_wait_group<1>();
     else
       ptx::cp_async_wait_group<0>();
-    const uint32_t* base = ring + (quads ? ((n % P) * (W / 4) * NT + tid) * 4 : (n % P) * W * NT + tid);
+    __syncwarp();
+    const uint32_t* row = ring + ((n % P) * NW + warp) * 32 * W + lane * W;
     if (quads) {
 #pragma unroll
       for (int q = 0; q < MW / 4; ++q) {
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (4 * q < W) v = reinterpret_cast<const uint4*>(base)[q * NT];
+        if (q < QR) v = reinterpret_cast<const uint4*>(row)[qpos(q, lane)];
         r[4 * q] = v.x;
         r[4 * q + 1] = v.y;
         r[4 * q + 2] = v.z;
@@ -246,10 +272,10 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       }
     } else {
 #pragma unroll
-      for (int w = 0; w < MW; ++w) r[w] = w < W ? base[w * NT] : 0u;
+      for (int w = 0; w < MW; ++w) r[w] = w < W ? row[w] : 0u;
     }
   };
-  if (nround > 0) prime(true, t.kbeg, rows_of(round_keys(0)));
+  if (nround > 0) prime(true, t.kbeg, round_keys(0));
 
   // ---- atom rows: chunks of `chunk` atoms through two buffers in the logit
   // store region, by bulk copies completing on bar0 / bar1. A chunk's copy is
@@ -441,6 +467,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
 #pragma unroll 1
     for (int i = 0; i < mine; ++i) {
       const int j = tid + i * NT;
+      const bool live = j < nk;
       uint32_t kw[MW];
       fetch(2 * i, kw);
       float s[HMAX];
@@ -450,7 +477,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       for (int w = 0; w < MW; ++w) {
         const int idx = static_cast<int>(kw[w] >> 16);
         const bool in = idx < NA;
-        bad |= !in;
+        bad |= live && !in;
         const float cf = in ? code_coeff(kw[w]) : 0.f;
         // an atom's logits of all heads sit side by side: 16-byte loads when
         // heads_per_kv is a multiple of 4
@@ -471,13 +498,14 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
             if (h < hpk) s[h] = fmaf(cf, row[h], s[h]);
         }
       }
-      issue(true, kb, mine, 2 * i + P);          // the K row's slot is free
+      issue(true, kb, nk, 2 * i + P);            // the K row's slot is free
       uint32_t vw[MW];
       fetch(2 * i + 1, vw);
       float csum = 0.f;                          // sum of |V coefficient| of the key
 #pragma unroll
       for (int w = 0; w < MW; ++w) csum += fabsf(code_coeff(vw[w]));
-      issue(true, kb, mine, 2 * i + 1 + P);      // the V row's slot is free
+      issue(true, kb, nk, 2 * i + 1 + P);        // the V row's slot is free
+      if (!live) continue;
       cs[j] = csum;
       const float bb = bias2(a, t, kb + j);
       float* dst = lg + j * hpk;
@@ -495,7 +523,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
 #pragma unroll
       for (int h = 0; h < HMAX; ++h) tmax[h] = fmaxf(tmax[h], s[h] + bb);
     }
-    prime(false, kb, mine);          // pass C's V rows come in across the barrier
+    prime(false, kb, nk);            // pass C's V rows come in across the barrier
     // this thread's bound relative to its own maxima, from its keys' logits
     // and coefficient sums (no copy involved)
     float tb[HMAX];
@@ -504,6 +532,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
 #pragma unroll 2
     for (int i = 0; i < mine; ++i) {
       const int j = tid + i * NT;
+      if (j >= nk) break;
       float l[HMAX];
       load_heads(lg + j * hpk, l);
       const float c = cs[j];
@@ -551,6 +580,10 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       const int j = tid + i * NT;
       uint32_t vw[MW];
       fetch(i, vw);
+      if (j >= nk) {                 // past the round: the warp's copies and syncs only
+        issue(false, kb, nk, i + P);
+        continue;
+      }
       float l[HMAX], ps[HMAX];       // weights in fixed-point units
       load_heads(lg + j * hpk, l);
 #pragma unroll
@@ -576,10 +609,10 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
         for (int h = 0; h < HMAX; ++h)
           if (h < hpk) atomicAdd(wrow + h * NA, static_cast<uint32_t>(__float2int_rn(ps[h] * cf)));
       }
-      issue(false, kb, mine, i + P);
+      issue(false, kb, nk, i + P);
     }
     // the next round's rows start coming in across the barrier
-    if (rd + 1 < nround) prime(true, kb + KR, rows_of(round_keys(rd + 1)));
+    if (rd + 1 < nround) prime(true, kb + KR, round_keys(rd + 1));
     __syncthreads();                 // the round's atomics done
     // fold: Wt and Wb relative to the new running maximum; Wb cleared
 #pragma unroll
