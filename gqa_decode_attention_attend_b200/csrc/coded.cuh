@@ -126,10 +126,11 @@ __device__ __forceinline__ void cta_reduce_heads(const float (*v)[NW], int hpk, 
 // value epilogue (threads own 4 columns of one head for a share of the atoms,
 // then the shares add in a fixed order).
 // Keys go in rounds of KR (a multiple of 512); thread tid takes keys tid, tid
-// + 512, ... of a round. Its code rows pass through its own P-row ring
-// (cp.async; no thread touches another's slots, and the next pass's first rows
-// are issued before each barrier, so they run across it). Per round, two
-// passes and one barrier between them:
+// + 512, ... of a round. Code rows pass through a P-row ring by cp.async, each
+// warp copying its 32 keys' rows together in whole 32-byte sectors into its
+// own part of a slot (the next pass's first rows are issued before each
+// barrier, so they run across it). Per round, two passes and one barrier
+// between them:
 //   A. the K and V rows of each key in turn: logits by table lookups into the
 //      round's logit store, each key's sum of |V coefficient|, and the
 //      thread's maxima per head; then, out of its own keys' entries of the
