@@ -163,6 +163,11 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   __shared__ float red2[HMAX][NW];       // per head, per warp: weight bounds
   __shared__ float smM[16], smL[16], smC[16];
   __shared__ float hM[16], hL[16];       // per head: base-2 running maximum, partition
+  // Above 8 heads the per-head values every thread shares (running maximum,
+  // the round's weight maximum, scale and rescale factor) live here, set by
+  // one thread per head, instead of in every thread's registers.
+  constexpr bool SH = HMAX > 8;
+  __shared__ float cM[HMAX], cMn[HMAX], cSc[HMAX], cFr[HMAX];
   __shared__ int smFlag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hpk = a.hpk, NA = c.n_atoms, W = c.words;
@@ -427,6 +432,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
     mrun[h] = -INFINITY;
     lthr[h] = 0.f;
   }
+  if (SH && tid < HMAX) cM[tid] = -INFINITY;   // read after the first round's barrier
   // (maximum, bound) pairs: the bound rescaled to the larger maximum; the
   // combination is symmetric, so a butterfly leaves the same bits in every lane
   auto pair_combine = [](float& m, float& s, float m2, float s2) {
@@ -556,8 +562,27 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
     __syncthreads();                 // red, red2 complete
     // ---- pass C
     float mn[HMAX], scale[HMAX], fr[HMAX];
+    if (SH) {
+      // thread h combines head h's pairs over the warps in order
+      if (tid < hpk) {
+        const int h = tid;
+        float m = red[h][0], sb = red2[h][0];
+        for (int w = 1; w < NW; ++w) pair_combine(m, sb, red[h][w], red2[h][w]);
+        const float mold = cM[h];
+        const float mnew = fmaxf(mold, m);
+        cFr[h] = (mnew == -INFINITY) ? 1.f : exp2f(mold - mnew);
+        cM[h] = mnew;
+        cSc[h] = block_weight_scale(m == -INFINITY ? 0.f : sb * exp2f(m - mnew));
+        cMn[h] = mnew == -INFINITY ? 0.f : mnew;
+      }
+      __syncthreads();               // cFr, cSc, cMn set
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h)
+        if (h < hpk) lthr[h] *= cFr[h];
+    }
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
+      if (SH) break;
       mn[h] = 0.f;
       scale[h] = 0.f;
       fr[h] = 1.f;
@@ -591,9 +616,9 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       for (int h = 0; h < HMAX; ++h) {
         ps[h] = 0.f;
         if (h < hpk) {
-          const float p = exp2f(l[h] - mn[h]);
+          const float p = exp2f(l[h] - (SH ? cMn[h] : mn[h]));
           lthr[h] += p;
-          ps[h] = p * scale[h];
+          ps[h] = p * (SH ? cSc[h] : scale[h]);
         }
       }
       // every word adds its weights, zero ones included (no branch); an index
@@ -619,9 +644,10 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
       if (h >= hpk) break;
-      const float u = scale[h] > 0.f ? 1.f / scale[h] : 0.f;
+      const float sch = SH ? cSc[h] : scale[h], frh = SH ? cFr[h] : fr[h];
+      const float u = sch > 0.f ? 1.f / sch : 0.f;
       for (int i = h * NA + tid; i < (h + 1) * NA; i += NT) {
-        Wt[i] = fmaf(Wt[i], fr[h], static_cast<float>(static_cast<int32_t>(Wb[i])) * u);
+        Wt[i] = fmaf(Wt[i], frh, static_cast<float>(static_cast<int32_t>(Wb[i])) * u);
         Wb[i] = 0u;
       }
     }
@@ -643,7 +669,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
 #pragma unroll
     for (int h = 0; h < HMAX; ++h)
       if (h < hpk && tid == h) {
-        hM[h] = mrun[h];
+        hM[h] = SH ? cM[h] : mrun[h];
         hL[h] = L[h];
       }
   }
