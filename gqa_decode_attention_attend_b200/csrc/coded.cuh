@@ -281,8 +281,6 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       for (int w = 0; w < MW; ++w) r[w] = w < W ? row[w] : 0u;
     }
   };
-  if (nround > 0) prime(true, t.kbeg, round_keys(0));
-
   // ---- atom rows: chunks of `chunk` atoms through two buffers in the logit
   // store region, by bulk copies completing on bar0 / bar1. A chunk's copy is
   // issued once every thread is done with the buffer (a barrier, and a proxy
@@ -292,6 +290,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   uint32_t phase0 = 0u, phase1 = 0u;
   float* abuf = lg;
   const int region = KR * (hpk + 1);                  // words of lg + cs (free outside rounds)
+  const int vwords = P * W * NT + KR * coded_key_words(W, hpk);   // ring + round region: V atom staging
   auto issue_atoms = [&](const float* atoms, int a0, int n, int b, float* base) {
     if (tid == 0 && n > 0) {
       const uint32_t bb = b ? bar1 : bar0;
@@ -316,14 +315,23 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   };
   // Run body(chunk start, count, rows) over all atoms of `atoms`, two chunks in flight.
   bool ok = true;
-  auto over_atoms = [&](const float* atoms, float* base, int words, auto&& body) {
+  // The first two chunks' copies (thread 0), into buffers nobody uses any more.
+  auto start_atoms = [&](const float* atoms, float* base, int words) {
+    const int chunk = words / 2 / D;
+    issue_atoms(atoms, 0, min(chunk, NA), 0, base);
+    if (NA > chunk) issue_atoms(atoms, chunk, min(chunk, NA - chunk), 1, base + static_cast<size_t>(chunk) * D);
+  };
+  // started: start_atoms has run already (else every thread's accesses to the
+  // buffers are fenced and waited for here first)
+  auto over_atoms = [&](const float* atoms, float* base, int words, bool started, auto&& body) {
     const int chunk = words / 2 / D;                   // atoms per buffer
     float* const buf1 = base + static_cast<size_t>(chunk) * D;
     const int nchunk = (NA + chunk - 1) / chunk;
-    ptx::fence_proxy_async_smem();
-    __syncthreads();
-    issue_atoms(atoms, 0, min(chunk, NA), 0, base);
-    if (nchunk > 1) issue_atoms(atoms, chunk, min(chunk, NA - chunk), 1, buf1);
+    if (!started) {
+      ptx::fence_proxy_async_smem();
+      __syncthreads();
+      start_atoms(atoms, base, words);
+    }
     for (int k = 0; k < nchunk && ok; ++k) {
       const int b = k & 1;
       float* const bufk = b ? buf1 : base;
@@ -338,6 +346,10 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
     }
   };
 
+  // The logit table's first atom rows are on their way (the logit store is
+  // untouched so far) before the first code rows are requested.
+  start_atoms(c.k_atoms, abuf, region);
+  if (nround > 0) prime(true, t.kbeg, round_keys(0));
   for (int i = tid; i < hpk * NA; i += NT) {
     Wt[i] = 0.f;
     Wb[i] = 0u;
@@ -367,7 +379,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
         }
     };
     load_q(0);
-    over_atoms(c.k_atoms, abuf, region, [&](int c0, int n, const float* rows) {
+    over_atoms(c.k_atoms, abuf, region, true, [&](int c0, int n, const float* rows) {
 #pragma unroll 1
       for (int h0 = 0; h0 < hpk; h0 += HT) {
         if (hpk > HT) load_q(h0);
@@ -637,9 +649,14 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       }
       issue(false, kb, nk, i + P);
     }
-    // the next round's rows start coming in across the barrier
-    if (rd + 1 < nround) prime(true, kb + KR, round_keys(rd + 1));
+    // the next round's rows start coming in across the barrier; after the
+    // last round, the V atoms' first chunks do (ring and store are free then)
+    if (rd + 1 < nround)
+      prime(true, kb + KR, round_keys(rd + 1));
+    else
+      ptx::fence_proxy_async_smem();
     __syncthreads();                 // the round's atomics done
+    if (rd + 1 == nround) start_atoms(c.v_atoms, reinterpret_cast<float*>(ring), vwords);
     // fold: Wt and Wb relative to the new running maximum; Wb cleared
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) {
@@ -688,7 +705,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   const int qd = tid % Q, hh = (tid / Q) % HMAX, ag = tid / (Q * HMAX);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (ok)
-    over_atoms(c.v_atoms, reinterpret_cast<float*>(ring), P * W * NT + KR * coded_key_words(W, hpk),
+    over_atoms(c.v_atoms, reinterpret_cast<float*>(ring), vwords, true,
                [&](int c0, int n, const float* rows) {
                  if (hh < hpk) {
                    const float* wr = Wt + hh * NA + c0;
