@@ -137,3 +137,27 @@ def test_coded_at_the_table_limit(D):
     ka2 = np.concatenate([ka, ka[:1]])
     with pytest.raises(gqa.GqaError):
         run_coded(w, kc, vc, ka2, ka2, dev, out_dtype=torch.float32)
+
+
+def test_coded_many_heads_rounds_and_bias():
+    """16 query heads per KV head (the values every thread shares then live in
+    shared memory), three rounds of keys on the longest sequence (one split of
+    2600 keys, rounds of 1024), and a bias row: finite values, and -inf over the
+    first 1100 keys of sequence 0, so that its first round is masked out
+    entirely and its second in part."""
+    dev = gu.device()
+    D, H, G, words, NA = 128, 32, 2, 8, 256
+    lengths = [2600, 1, 1100]
+    w = workloads.make("cbias", lengths, H, G, D, dtype=torch.float32, seed=14, carry=True)
+    kc, vc, ka, va = make_codes(w.total_rows, G, words, NA, D, seed=15)
+    rng = np.random.default_rng(16)
+    bias = rng.normal(0, 1, w.total_rows).astype(np.float32)
+    off = w.offsets.numpy()
+    bias[off[0]:off[0] + 1100] = -np.inf
+    ref = oracle.coded_decode_attend(workloads.host_array(w.q), kc, vc, ka, va, off, H, G,
+                                     carry=tuple(t.numpy() for t in w.carry), bias=bias)
+    for ns in (0, 1):
+        out = run_coded(w, kc, vc, ka, va, dev, out_dtype=torch.float32, num_splits=ns,
+                        bias=torch.from_numpy(bias).to(dev))
+        gu.assert_close(out.reshape(-1, D).cpu().numpy(), ref.out, torch.float32,
+                        f"coded 16 heads per KV head, rounds, bias, splits{ns}")
