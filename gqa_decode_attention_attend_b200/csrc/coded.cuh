@@ -81,14 +81,14 @@ __device__ __forceinline__ float code_coeff(uint32_t word) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(word & 0xFFFFu)));
 }
 
-// Fixed-point scale of one head's value weights in a block. The weights of
-// any atom sum, in absolute value, to at most bound = sum_j p_j sum_w |c_jw|
-// over the block's keys, so weights scaled by 2^e with bound * 2^e <= 2^30
-// (and each rounded by at most 1/2) sum without overflow in 32-bit integers;
-// the rounding errors stay below 2^-30 * bound per weight, relative to the
-// block's whole value sum.
-__device__ __forceinline__ float block_weight_scale(float bound) {
-  if (!(bound > 0.f)) return 1073741824.f;                   // no weight this block (or NaN)
+// Fixed-point scale of one head's value weights in a round of keys. The
+// weights of any atom sum, in absolute value, to at most bound = sum_j p_j
+// sum_w |c_jw| over the round's keys, so weights scaled by 2^e with
+// bound * 2^e <= 2^30 (and each rounded by at most 1/2) sum without overflow
+// in 32-bit integers. The chosen e puts bound * 2^e in (2^29, 2^30], so the
+// rounding error of a weight (half a unit, 2^-e / 2) stays below 2^-30 * bound.
+__device__ __forceinline__ float round_weight_scale(float bound) {
+  if (!(bound > 0.f)) return 1073741824.f;                   // no weight this round (or NaN)
   if (!(bound < INFINITY)) return 0.f;
   // ceil(log2(bound)) from the bits: the exponent, plus one unless a power of 2
   const int bits = __float_as_int(bound);
@@ -584,7 +584,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
         const float mnew = fmaxf(mold, m);
         cFr[h] = (mnew == -INFINITY) ? 1.f : exp2f(mold - mnew);
         cM[h] = mnew;
-        cSc[h] = block_weight_scale(m == -INFINITY ? 0.f : sb * exp2f(m - mnew));
+        cSc[h] = round_weight_scale(m == -INFINITY ? 0.f : sb * exp2f(m - mnew));
         cMn[h] = mnew == -INFINITY ? 0.f : mnew;
       }
       __syncthreads();               // cFr, cSc, cMn set
@@ -610,7 +610,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       lthr[h] *= fr[h];
       // weights relative to the running maximum are at most those relative
       // to the round's, so the round's bound still bounds them
-      scale[h] = block_weight_scale(m == -INFINITY ? 0.f : sb * exp2f(m - mnew));
+      scale[h] = round_weight_scale(m == -INFINITY ? 0.f : sb * exp2f(m - mnew));
       mn[h] = mnew == -INFINITY ? 0.f : mnew;    // all masked so far: weights 0
     }
 #pragma unroll 1

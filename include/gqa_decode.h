@@ -240,7 +240,7 @@ typedef struct {
  * device error word. The per-atom value weights are summed per round of keys (a
  * multiple of 512, at most 8192, as many as shared memory holds) in 32-bit fixed
  * point, scaled by a power of two to the round's largest possible sum
- * sum_j p_j sum_w |coeff_jw| (rounding error at most 2^-31 of it per weight), so
+ * sum_j p_j sum_w |coeff_jw| (rounding error below 2^-30 of it per weight), so
  * results are bit-reproducible. The split plan is the coded kernel's own (one
  * CTA of 512 threads per SM), so size the workspace with
  * gqa_decode_coded_workspace_size. */

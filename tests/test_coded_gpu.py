@@ -96,7 +96,7 @@ def test_coded_is_deterministic():
 def test_coded_sharp_softmax_and_wide_coefficients(words):
     """Peaked logits (score scale 1 instead of 1/sqrt(128): few keys carry the
     weight) and coefficients spread over four and a half orders of magnitude,
-    at the fp32 tolerance: the fixed-point scale of each block follows the
+    at the fp32 tolerance: the fixed-point scale of each round follows the
     weights actually present."""
     dev = gu.device()
     D, H, G, NA = 128, 16, 4, 96
