@@ -149,7 +149,8 @@ __device__ __forceinline__ void cta_reduce_heads(const float (*v)[NW], int hpk, 
 // results are bit-reproducible. A segment with one split (the tile is the
 // whole sequence) folds the carry and writes out / state_out directly; others
 // go through the same partial states and fused merge as the other partition
-// kernels. MW: a compile-time bound on the words per row (4, 8 or 16).
+// kernels. HMAX: a compile-time bound on heads_per_kv (4, 8 or 16); MW: on
+// the words per row (4, 8 or 16).
 template <int D, int HMAX, int MW>
 __global__ void __launch_bounds__(kCodedThreads, 1)
 gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
