@@ -123,8 +123,8 @@ __device__ __forceinline__ void cta_reduce_heads(const float (*v)[NW], int hpk, 
 // One CTA of 512 threads per SM. Atom rows come into shared memory by TMA bulk
 // copies, two chunks in flight, for the logit table (warps take atoms, lanes
 // across D, a warp reduce-scatter sums the partial dot products) and for the
-// value epilogue (threads own 4 columns of one head for a share of the atoms,
-// then the shares add in a fixed order).
+// value epilogue (threads own 4 columns of up to 4 heads for a share of the
+// atoms, then the shares add in a fixed order).
 // Keys go in rounds of KR (a multiple of 512); thread tid takes keys tid, tid
 // + 512, ... of a round. Code rows pass through a P-row ring by cp.async, each
 // warp copying its 32 keys' rows together in whole 32-byte sectors into its
@@ -696,47 +696,61 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   if (threadIdx.x == 0) ptx::grid_launch_dependents();
 
   // acc[h][d] = sum over atoms of Wt[h][atom] * vatom[atom][d]: the V atoms
-  // come through the round region (and the ring) in chunks. Thread tid owns
-  // column quad qd = tid % Q of head h = (tid / Q) % HMAX for atom share ag =
-  // tid / (Q * HMAX) (atoms ag, ag + AG, ...), summing its atoms in order; the
-  // AG shares then add in order.
+  // come through the ring and round region in chunks. Thread tid owns column
+  // quad qd = tid % Q of the HG heads hg * HG .. hg * HG + HG - 1 (hg = (tid /
+  // Q) % NG) for atom share ag = tid / (Q * NG) (atoms ag, ag + AG, ...): it
+  // reads an atom's quad once for its HG heads and sums its atoms in order.
+  // Then thread (qd, hg, ag < HG) adds head hg * HG + ag over the AG shares in
+  // order.
   constexpr int Q = D / 4;
-  constexpr int AG = NT / (Q * HMAX);                  // atom shares: 1 .. 8
-  static_assert(AG >= 1 && Q * HMAX * AG == NT, "threads cover quads x heads x shares");
-  const int qd = tid % Q, hh = (tid / Q) % HMAX, ag = tid / (Q * HMAX);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int HG = HMAX < 4 ? HMAX : 4;              // heads per thread
+  constexpr int NG = HMAX / HG;                        // head groups
+  constexpr int AG = NT / (Q * NG);                    // atom shares: 4 .. 32
+  static_assert(Q * NG * AG == NT && AG >= HG, "threads cover quads x head groups x shares");
+  // the shares' sums, NT x HG float4, fit the V staging region: it is at least
+  // the free words less the largest tables and one 512-key round's rounding
+  static_assert(coded_free_words() - 3 * kCodedMaxTableEntries - kCodedThreads * (16 + 1) >= NT * HG * 4,
+                "the shares' sums fit the V staging region");
+  const int qd = tid % Q, hg = (tid / Q) % NG, ag = tid / (Q * NG);
+  float4 acc4[HG];
+#pragma unroll
+  for (int k = 0; k < HG; ++k) acc4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (ok)
     over_atoms(c.v_atoms, reinterpret_cast<float*>(ring), vwords, true,
                [&](int c0, int n, const float* rows) {
-                 if (hh < hpk) {
-                   const float* wr = Wt + hh * NA + c0;
-#pragma unroll 4
+                 if (hg * HG < hpk) {
+                   const float* wr = Wt + hg * HG * NA + c0;
+#pragma unroll 2
                    for (int at = ag; at < n; at += AG) {
                      const float4 vv = *reinterpret_cast<const float4*>(rows + at * D + qd * 4);
-                     const float wgt = wr[at];
-                     acc.x = fmaf(wgt, vv.x, acc.x);
-                     acc.y = fmaf(wgt, vv.y, acc.y);
-                     acc.z = fmaf(wgt, vv.z, acc.z);
-                     acc.w = fmaf(wgt, vv.w, acc.w);
+#pragma unroll
+                     for (int k = 0; k < HG; ++k) {
+                       const float wgt = hg * HG + k < hpk ? wr[k * NA + at] : 0.f;
+                       acc4[k].x = fmaf(wgt, vv.x, acc4[k].x);
+                       acc4[k].y = fmaf(wgt, vv.y, acc4[k].y);
+                       acc4[k].z = fmaf(wgt, vv.z, acc4[k].z);
+                       acc4[k].w = fmaf(wgt, vv.w, acc4[k].w);
+                     }
                    }
                  }
                });
   if (!ok) return;                   // a copy never landed (flagged): no state out
   __syncthreads();                   // the atom buffers are free
-  if (AG > 1) {
-    float4* sh = reinterpret_cast<float4*>(ring);      // [AG][HMAX][Q] (the region holds >= 8 KB)
-    sh[(ag * HMAX + hh) * Q + qd] = acc;
-    __syncthreads();
-    if (ag == 0)
-      for (int g2 = 1; g2 < AG; ++g2) {
-        const float4 o = sh[(g2 * HMAX + hh) * Q + qd];
-        acc.x += o.x;
-        acc.y += o.y;
-        acc.z += o.z;
-        acc.w += o.w;
-      }
-  }
-  const bool owner = ag == 0 && hh < hpk;
+  float4* sh = reinterpret_cast<float4*>(ring);        // [AG][NG][HG][Q]
+#pragma unroll
+  for (int k = 0; k < HG; ++k) sh[((ag * NG + hg) * HG + k) * Q + qd] = acc4[k];
+  __syncthreads();
+  const int hh = hg * HG + ag;                          // this thread's head of the sum (ag < HG)
+  const bool owner = ag < HG && hh < hpk;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (owner)
+    for (int g2 = 0; g2 < AG; ++g2) {
+      const float4 o = sh[((g2 * NG + hg) * HG + ag) * Q + qd];
+      acc.x += o.x;
+      acc.y += o.y;
+      acc.z += o.z;
+      acc.w += o.w;
+    }
 
   // The state goes out as store_partial writes a single slot (m in natural-log units).
   if (owner) *reinterpret_cast<float4*>(a.part_acc + state_index(a, t, hh) * D + qd * 4) = acc;
