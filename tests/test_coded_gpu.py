@@ -161,3 +161,19 @@ def test_coded_many_heads_rounds_and_bias():
                         bias=torch.from_numpy(bias).to(dev))
         gu.assert_close(out.reshape(-1, D).cpu().numpy(), ref.out, torch.float32,
                         f"coded 16 heads per KV head, rounds, bias, splits{ns}")
+
+
+def test_coded_long_single_split_over_rounds():
+    """8 words, 256 atoms, 4 heads per KV head (rounds of 6656 keys): one split
+    of 14000 keys takes three rounds, the last one ragged, beside a short
+    sequence; the planned splits as well."""
+    dev = gu.device()
+    D, H, G, words, NA = 128, 32, 8, 8, 256
+    w = workloads.make("clong", [14000, 130], H, G, D, dtype=torch.bfloat16, seed=17, carry=True)
+    kc, vc, ka, va = make_codes(w.total_rows, G, words, NA, D, seed=18)
+    ref = oracle.coded_decode_attend(workloads.host_array(w.q), kc, vc, ka, va, w.offsets.numpy(), H, G,
+                                     carry=tuple(t.numpy() for t in w.carry))
+    for ns in (1, 0):
+        out = run_coded(w, kc, vc, ka, va, dev, out_dtype=torch.float32, num_splits=ns)
+        gu.assert_close(out.reshape(-1, D).cpu().numpy(), ref.out, torch.float32,
+                        f"coded long single split, splits{ns}")
