@@ -40,7 +40,8 @@ def run_coded(w, kc, vc, ka, va, dev, **kw):
 
 
 @pytest.mark.parametrize("D,H,G,words,n_atoms", [(128, 32, 8, 8, 256), (64, 16, 2, 4, 1024),
-                                                 (128, 16, 1, 1, 64), (128, 48, 8, 16, 512)])
+                                                 (128, 16, 1, 1, 64), (128, 48, 8, 16, 512),
+                                                 (64, 16, 4, 4, 512)])
 @pytest.mark.parametrize("qdt", [torch.bfloat16, torch.float32], ids=["bf16q", "f32q"])
 def test_coded_attention(D, H, G, words, n_atoms, qdt):
     dev = gu.device()
