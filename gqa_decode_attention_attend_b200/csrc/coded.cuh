@@ -150,8 +150,9 @@ __device__ __forceinline__ void cta_reduce_heads(const float (*v)[NW], int hpk, 
 // whole sequence) folds the carry and writes out / state_out directly; others
 // go through the same partial states and fused merge as the other partition
 // kernels. HMAX: a compile-time bound on heads_per_kv (4, 8 or 16); MW: on
-// the words per row (4, 8 or 16); EXACT: the rows have exactly MW words, so
-// that the word count and everything derived from it are constants.
+// the words per row (4, 8 or 16); EXACT: the rows have exactly MW words and
+// heads_per_kv is HMAX, so that both counts and everything derived from them
+// are constants.
 template <int D, int HMAX, int MW, bool EXACT = false>
 __global__ void __launch_bounds__(kCodedThreads, 1)
 gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
@@ -172,7 +173,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   __shared__ float cM[HMAX], cMn[HMAX], cSc[HMAX], cFr[HMAX];
   __shared__ int smFlag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int hpk = a.hpk, NA = c.n_atoms, W = EXACT ? MW : c.words;
+  const int hpk = EXACT ? HMAX : a.hpk, NA = c.n_atoms, W = EXACT ? MW : c.words;
   const int P = coded_ring_rows(W, hpk, NA);
   const int KR = coded_round_keys(W, hpk, NA);
   const uint32_t bar0 = ptx::smem_u32(dsm);                    // atom copies into buffer 0 / 1

@@ -71,9 +71,10 @@ static_assert(gqa::coded_ring_fits(1, gqa::kMaxCodeWords, 1, gqa::kCodedMaxTable
                   gqa::coded_ring_fits(1, gqa::kMaxCodeWords, 16, gqa::kCodedMaxTableEntries / 16),
               "the largest coded tables fit beside a ring row and the smallest round store");
 
-// Bounds that also have a variant for rows of exactly MW words (its constant
-// word count saves the key loop's guards: 38.5 -> 36.2 us a call on 16 x 4096
-// keys, 8 words, measured on B200); the others would spill more registers.
+// Bounds that also have a variant for exactly HMAX heads per KV head and MW
+// words per row (its constant counts save the loops' guards: 38.5 -> 36.2 us
+// a call on 16 x 4096 keys, 8 words, measured on B200); the others would
+// spill more registers.
 template <int HMAX, int MW>
 constexpr bool kCodedExact = HMAX == 4 && MW <= 8;
 
@@ -463,8 +464,9 @@ cudaError_t launch_f32(const PartitionArgs& a, unsigned grid, cudaStream_t st, b
 // The coded kernel for heads_per_kv bound hp (4, 8, 16) and words bound mw (4, 8, 16).
 template <int D, int HMAX>
 cudaError_t launch_coded_hp(Launch& l, int mw, const PartitionArgs& a, const gqa::CodedArgs& c) {
-  // rows of exactly the bound's words take the variant compiled for them
-  const bool ex = c.words == mw;
+  // rows of exactly the bound's words, with the bound's heads per KV head,
+  // take the variant compiled for them
+  const bool ex = c.words == mw && a.hpk == HMAX;
   if (mw == 4) {
     if constexpr (kCodedExact<HMAX, 4>)
       if (ex) return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 4, true>, a, c);
