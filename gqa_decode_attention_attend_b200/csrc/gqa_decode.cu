@@ -71,12 +71,13 @@ static_assert(gqa::coded_ring_fits(1, gqa::kMaxCodeWords, 1, gqa::kCodedMaxTable
                   gqa::coded_ring_fits(1, gqa::kMaxCodeWords, 16, gqa::kCodedMaxTableEntries / 16),
               "the largest coded tables fit beside a ring row and the smallest round store");
 
-// Bounds that also have a variant for exactly HMAX heads per KV head and MW
-// words per row (its constant counts save the loops' guards: 38.5 -> 36.2 us
-// a call on 16 x 4096 keys, 8 words, measured on B200); the others would
-// spill more registers.
+// Every bound also has a variant for exactly HMAX heads per KV head and MW
+// words per row: its constant counts fold the loops' guards (on 16 x 4096
+// keys, 4 heads, 8 words: 38.5 -> 33.9 us a call, measured on B200) and spill
+// as much or less than the general one at most bounds. The switch stays per
+// bound.
 template <int HMAX, int MW>
-constexpr bool kCodedExact = HMAX == 4 && MW <= 8;
+constexpr bool kCodedExact = true;
 
 template <int D, int HMAX, int MW>
 cudaError_t prepare_coded() {
@@ -477,6 +478,8 @@ cudaError_t launch_coded_hp(Launch& l, int mw, const PartitionArgs& a, const gqa
       if (ex) return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 8, true>, a, c);
     return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 8>, a, c);
   }
+  if constexpr (kCodedExact<HMAX, 16>)
+    if (ex) return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 16, true>, a, c);
   return cudaLaunchKernelEx(&l.cfg, gqa::gqa_partition_coded_kernel<D, HMAX, 16>, a, c);
 }
 
