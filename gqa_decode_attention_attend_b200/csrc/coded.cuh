@@ -352,7 +352,11 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   // The logit table's first atom rows are on their way (the logit store is
   // untouched so far) before the first code rows are requested.
   start_atoms(c.k_atoms, abuf, region);
-  if (nround > 0) prime(true, t.kbeg, round_keys(0));
+  // the first two rows before the table, the rest after it: issuing copies
+  // holds a warp, and the table should start as soon as its atoms land
+  const int early_rows = P < 2 ? P : 2;
+  if (nround > 0)
+    for (int n = 0; n < early_rows; ++n) issue(true, t.kbeg, round_keys(0), n);
   for (int i = tid; i < hpk * NA; i += NT) {
     Wt[i] = 0.f;
     Wb[i] = 0u;
@@ -428,6 +432,8 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
       }
     });
   }
+  if (nround > 0)
+    for (int n = early_rows; n < P; ++n) issue(true, t.kbeg, round_keys(0), n);
   __syncthreads();                   // the table is complete; the logit store is free
 
   // Running maximum per head (identical in every thread) and this thread's
