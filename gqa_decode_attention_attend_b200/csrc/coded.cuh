@@ -318,16 +318,23 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   };
   // Run body(chunk start, count, rows) over all atoms of `atoms`, two chunks in flight.
   bool ok = true;
+  // Atoms per buffer: as many as half the words hold, a multiple of 128 when
+  // that many fit (the table's 16 warps take 8 atoms a step, so a chunk of
+  // 130 would leave one warp a second step for 2 atoms).
+  auto atoms_per_chunk = [&](int words) {
+    const int n = words / 2 / D;
+    return n >= 128 ? n / 128 * 128 : n;
+  };
   // The first two chunks' copies (thread 0), into buffers nobody uses any more.
   auto start_atoms = [&](const float* atoms, float* base, int words) {
-    const int chunk = words / 2 / D;
+    const int chunk = atoms_per_chunk(words);
     issue_atoms(atoms, 0, min(chunk, NA), 0, base);
     if (NA > chunk) issue_atoms(atoms, chunk, min(chunk, NA - chunk), 1, base + static_cast<size_t>(chunk) * D);
   };
   // started: start_atoms has run already (else every thread's accesses to the
   // buffers are fenced and waited for here first)
   auto over_atoms = [&](const float* atoms, float* base, int words, bool started, auto&& body) {
-    const int chunk = words / 2 / D;                   // atoms per buffer
+    const int chunk = atoms_per_chunk(words);           // atoms per buffer
     float* const buf1 = base + static_cast<size_t>(chunk) * D;
     const int nchunk = (NA + chunk - 1) / chunk;
     if (!started) {
