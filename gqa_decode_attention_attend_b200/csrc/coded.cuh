@@ -50,9 +50,10 @@ constexpr int kCodedMaxRoundKeys = 8192;
 //   tables  3 x hpk x n_atoms: logit table, value weights, round weights.
 __host__ __device__ constexpr int coded_table_words(int hpk, int n_atoms) { return 3 * hpk * n_atoms; }
 __host__ __device__ constexpr int coded_free_words() { return (kCodedSmemBudget - kCodedFixedBytes) / 4; }
-__host__ __device__ constexpr int coded_key_words(int words, int hpk) { return 0 * words + hpk + 1; }
+// words of the round region per key: its logits and its |V coefficient| sum
+__host__ __device__ constexpr int coded_key_words(int hpk) { return hpk + 1; }
 __host__ __device__ constexpr bool coded_ring_fits(int rows, int words, int hpk, int n_atoms) {
-  return rows * words * kCodedThreads + kCodedThreads * coded_key_words(words, hpk) +
+  return rows * words * kCodedThreads + kCodedThreads * coded_key_words(hpk) +
              coded_table_words(hpk, n_atoms) <=
          coded_free_words();
 }
@@ -63,7 +64,7 @@ __host__ __device__ constexpr int coded_ring_rows(int words, int hpk, int n_atom
 }
 __host__ __device__ constexpr int coded_round_keys_uncapped(int words, int hpk, int n_atoms) {
   return (coded_free_words() - coded_ring_rows(words, hpk, n_atoms) * words * kCodedThreads -
-          coded_table_words(hpk, n_atoms)) / coded_key_words(words, hpk) / kCodedThreads * kCodedThreads;
+          coded_table_words(hpk, n_atoms)) / coded_key_words(hpk) / kCodedThreads * kCodedThreads;
 }
 __host__ __device__ constexpr int coded_round_keys(int words, int hpk, int n_atoms) {
   return coded_round_keys_uncapped(words, hpk, n_atoms) > kCodedMaxRoundKeys
@@ -73,7 +74,7 @@ __host__ __device__ constexpr int coded_round_keys(int words, int hpk, int n_ato
 __host__ __device__ constexpr size_t coded_smem_bytes(int words, int hpk, int n_atoms) {
   return kCodedFixedBytes +
          4 * (static_cast<size_t>(coded_ring_rows(words, hpk, n_atoms)) * words * kCodedThreads +
-              static_cast<size_t>(coded_round_keys(words, hpk, n_atoms)) * coded_key_words(words, hpk) +
+              static_cast<size_t>(coded_round_keys(words, hpk, n_atoms)) * coded_key_words(hpk) +
               coded_table_words(hpk, n_atoms));
 }
 
@@ -293,7 +294,7 @@ gqa_partition_coded_kernel(const PartitionArgs a, const CodedArgs c) {
   uint32_t phase0 = 0u, phase1 = 0u;
   float* abuf = lg;
   const int region = KR * (hpk + 1);                  // words of lg + cs (free outside rounds)
-  const int vwords = P * W * NT + KR * coded_key_words(W, hpk);   // ring + round region: V atom staging
+  const int vwords = P * W * NT + KR * coded_key_words(hpk);   // ring + round region: V atom staging
   auto issue_atoms = [&](const float* atoms, int a0, int n, int b, float* base) {
     if (tid == 0 && n > 0) {
       const uint32_t bb = b ? bar1 : bar0;
