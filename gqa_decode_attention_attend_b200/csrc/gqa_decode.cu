@@ -540,6 +540,7 @@ PartitionArgs make_args(const gqa_decode_params* p, const Resolved& r, uint8_t* 
   }
   a.err = reinterpret_cast<uint32_t*>(ws);
   a.merge = r.want_merge ? 1 : 0;
+  a.partials_internal = r.has_partials ? 0 : 1;
   a.counters = r.want_merge ? reinterpret_cast<uint32_t*>(ws + r.off_counters) : nullptr;
   const bool has_carry = state_present(p->carry_in);
   a.cm = has_carry ? p->carry_in.m : nullptr;

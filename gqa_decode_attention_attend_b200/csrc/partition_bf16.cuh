@@ -374,6 +374,12 @@ gqa_partition_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   // state, but still takes its merge ticket, so that the segment's ticket
   // counter returns to zero as after any other call.
   const bool tile_aborted = *abort_flag != 0;
+  // The sequence's only split, with the partial states the call's own: the
+  // output straight from the slots above (no partial state stored, no ticket).
+  if (a.merge && a.partials_internal && !tile_aborted && t.kbeg == 0 && t.kend == t.n) {
+    finalize_single_split<D, W, HP>(a, t, ms, ls, accs, nslots, ctid, smM, smL, smC, smN, NamedSync128{});
+    return;
+  }
   if (!tile_aborted) store_partial<D, W, HP>(a, t, ms, ls, accs, ctid, 32 * W, nslots);
   static_assert(C::kConsumerWarps == 4, "NamedSync128 spans the four consumer warps");
   if (a.merge) {

@@ -61,6 +61,9 @@ struct PartitionArgs {
   // launches): 1 = once its producer has issued the tile's last load, 0 = once
   // its consumers have finished the tile's cache stream.
   int32_t trigger_at_last_load;
+  // The partial states are the call's own scratch (no partials_out): a tile
+  // that is its sequence's only split may then finalise without storing one.
+  int32_t partials_internal;
 };
 
 // Work item of a CTA: flattened index -> (b, split c, g), g fastest so that the
@@ -493,6 +496,98 @@ __device__ __forceinline__ bool merge_segment_smem(const PartitionArgs& a, const
       a.ol[row0 + h] = smL[h];
     }
   return true;
+}
+
+// A segment with one split, finalised by its CTA straight from the per-slot
+// states in shared memory (ms, ls [slots][HP] base-2; accs [slots][HP][D + 4]
+// rescaled to the tile maximum): store_partial's arithmetic followed by
+// merge_segment_smem's for one split and the carry, in the same order, without
+// the partial state's store and reload. Run by the 128 threads tid; smW holds
+// a per-head weight.
+template <int D, int W, int HP, class Sync>
+__device__ __forceinline__ void finalize_single_split(const PartitionArgs& a, const Tile& t, const float* ms,
+                                                      const float* ls, const float* accs, int nslots, int tid,
+                                                      float* smM, float* smL, float* smC, float* smW, Sync sync) {
+  constexpr int NT = 128, P = D + 4, Q = D / 4, GC = NT / Q;
+  const int hpk = a.hpk;
+  const size_t row0 = static_cast<size_t>(t.b) * a.H + static_cast<size_t>(t.g) * hpk;
+  for (int h = tid; h < hpk; h += NT) {
+    // the tile's state, as store_partial forms it
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < W + 1; ++w)
+      if (w < nslots) Mt = fmaxf(Mt, ms[w * HP + h]);
+    const float Mu = (Mt == -INFINITY) ? 0.f : Mt;
+    float Lt = 0.f;
+#pragma unroll
+    for (int w = 0; w < W + 1; ++w)
+      if (w < nslots) Lt += ls[w * HP + h] * exp2f(ms[w * HP + h] - Mu);
+    const float mt = (Lt == 0.f) ? -INFINITY : Mt * kLn2;
+    // one split and the carry, as merge_segment_smem folds them
+    const size_t r = row0 + h;
+    float M = (Lt != 0.f) ? mt : -INFINITY;
+    const bool has_carry = a.cl != nullptr && a.cl[r] != 0.f;
+    if (has_carry) M = fmaxf(M, a.cm[r]);
+    const float wt = (Lt != 0.f && M != -INFINITY) ? expf(mt - M) : 0.f;
+    float L = fmaf(Lt, wt, 0.f);
+    float wc = 0.f;
+    if (has_carry) {
+      wc = expf(a.cm[r] - M);
+      L = fmaf(a.cl[r], wc, L);
+    }
+    smM[h] = M;
+    smL[h] = L;
+    smC[h] = wc;
+    smW[h] = wt;
+  }
+  sync();
+  const int qd = tid % Q, hg = tid / Q;
+  for (int h = hg; h < hpk; h += GC) {
+    const size_t r = row0 + h;
+    float sv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < W + 1; ++w)
+        if (w < nslots) acc += accs[(w * HP + h) * P + qd * 4 + e];
+      sv[e] = acc;
+    }
+    const float wt = smW[h];
+    float4 y = make_float4(fmaf(sv[0], wt, 0.f), fmaf(sv[1], wt, 0.f), fmaf(sv[2], wt, 0.f), fmaf(sv[3], wt, 0.f));
+    const float cw = smC[h];
+    if (cw != 0.f) {
+      const float4 cv = *reinterpret_cast<const float4*>(a.cacc + r * D + qd * 4);
+      y.x = fmaf(cv.x, cw, y.x);
+      y.y = fmaf(cv.y, cw, y.y);
+      y.z = fmaf(cv.z, cw, y.z);
+      y.w = fmaf(cv.w, cw, y.w);
+    }
+    if (a.oacc) *reinterpret_cast<float4*>(a.oacc + r * D + qd * 4) = y;
+    if (a.out) {
+      const float L = smL[h];
+      const float o0 = (L == 0.f) ? 0.f : __fdiv_rn(y.x, L);
+      const float o1 = (L == 0.f) ? 0.f : __fdiv_rn(y.y, L);
+      const float o2 = (L == 0.f) ? 0.f : __fdiv_rn(y.z, L);
+      const float o3 = (L == 0.f) ? 0.f : __fdiv_rn(y.w, L);
+      if (a.out_bf16) {
+        __nv_bfloat162* dst =
+            reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.out) + r * D + qd * 4);
+        dst[0] = __floats2bfloat162_rn(o0, o1);
+        dst[1] = __floats2bfloat162_rn(o2, o3);
+      } else {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + r * D + qd * 4) = make_float4(o0, o1, o2, o3);
+      }
+    }
+  }
+  // m and l of the state out after every thread has read the carry (state out
+  // may alias it)
+  sync();
+  if (a.om)
+    for (int h = tid; h < hpk; h += NT) {
+      a.om[row0 + h] = (smL[h] == 0.f) ? -INFINITY : smM[h];
+      a.ol[row0 + h] = smL[h];
+    }
 }
 
 // After the CTA's partial state is stored: take a ticket on the segment and,
